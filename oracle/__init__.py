@@ -1,0 +1,175 @@
+"""CPU oracle for the BinaryAttention forward pass (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The CUDA
+product path never does, and the two share no code: this wrapper loads
+``ba_oracle.c`` (plain C, fp64), compiled with gcc into ``libba_oracle.so``.
+
+Source ("BA notes"): the paper-notes page "BinaryAttention: One-Bit
+QK-Attention for Vision and Diffusion Transformers" (CVPR 2026), sections
+Key design 1 (scaled binary Q/K), Key design 2 (bias enhancement) and Key
+design 3 (hybrid 8-bit quantisation of P and V).  Every numeric step lives in
+the C file; this module only marshals numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ba_oracle.c")
+_LIB = os.path.join(_HERE, "libba_oracle.so")
+_lib = None
+
+BIAS_NONE, BIAS_DENSE, BIAS_RELPOS2D = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile ba_oracle.c with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared",
+                               "-ffp-contract=off", "-fno-fast-math", "-D_GNU_SOURCE",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    i32, i64 = ctypes.c_int, ctypes.c_int64
+    lib.bao_words.argtypes = [i32]
+    lib.bao_words.restype = i32
+    lib.bao_pack.argtypes = [P, i64, i32, P, P]
+    lib.bao_pack.restype = None
+    lib.bao_dot_pm1.argtypes = [P, P, i32]
+    lib.bao_dot_pm1.restype = ctypes.c_int32
+    lib.bao_dot_bits.argtypes = [P, P, i32]
+    lib.bao_dot_bits.restype = ctypes.c_int32
+    lib.bao_scores.argtypes = [P, P, i64, i32, i32, P]
+    lib.bao_scores.restype = None
+    lib.bao_bias_value.argtypes = [i32, P, i64, i32, i32, i32, i32, i32, i32]
+    lib.bao_bias_value.restype = ctypes.c_double
+    lib.bao_quant_v.argtypes = [P, i64, i32, i32, P, P]
+    lib.bao_quant_v.restype = None
+    lib.bao_attention_rows.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32,
+                                       i32, i32, i32, i64, i32, i32, P, P, P, P]
+    lib.bao_attention_rows.restype = None
+    lib.bao_attention_fwd.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32,
+                                      i32, i32, i32, i32, P, i32]
+    lib.bao_attention_fwd.restype = i32
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def words(d: int) -> int:
+    return _load().bao_words(d)
+
+
+def pack(x):
+    """Sign bits [..., W] uint32 and per-token mean |x| [...] float64."""
+    x = _c(x, np.float32)
+    d = x.shape[-1]
+    T = x.size // d
+    W = words(d)
+    bits = np.zeros(x.shape[:-1] + (W,), np.uint32)
+    mu = np.zeros(x.shape[:-1], np.float64)
+    _load().bao_pack(_ptr(x), T, d, _ptr(bits), _ptr(mu))
+    return bits, mu
+
+
+def dot_pm1(q, k) -> int:
+    q, k = _c(q, np.float32), _c(k, np.float32)
+    return int(_load().bao_dot_pm1(_ptr(q), _ptr(k), q.shape[-1]))
+
+
+def dot_bits(a, b, d: int) -> int:
+    a, b = _c(a, np.uint32), _c(b, np.uint32)
+    return int(_load().bao_dot_bits(_ptr(a), _ptr(b), d))
+
+
+def scores(bq, bk, d: int):
+    """z [BH, N, N] int32 from bits [BH, N, W]."""
+    bq, bk = _c(bq, np.uint32), _c(bk, np.uint32)
+    BH, N = bq.shape[0], bq.shape[1]
+    z = np.zeros((BH, N, N), np.int32)
+    _load().bao_scores(_ptr(bq), _ptr(bk), BH, N, d, _ptr(z))
+    return z
+
+
+def bias_value(kind, bias, ld, h, N, gh, gw, i, j) -> float:
+    b = None if bias is None else _c(bias, np.float32)
+    return float(_load().bao_bias_value(kind, _ptr(b), ld, h, N, gh, gw, i, j))
+
+
+def quant_v(v):
+    """vq [BH, N, d] int8 and sv [BH, d] float32 from v [BH, N, d]."""
+    v = _c(v, np.float32)
+    BH, N, d = v.shape
+    vq = np.zeros((BH, N, d), np.int8)
+    sv = np.zeros((BH, d), np.float32)
+    _load().bao_quant_v(_ptr(v), BH, N, d, _ptr(vq), _ptr(sv))
+    return vq, sv
+
+
+def attention_rows(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw,
+                   H, bh, row_lo, row_hi, d, want_pq=False):
+    """Rows [row_lo, row_hi) of head bh; returns (out, pq, l, m)."""
+    bq, bk = _c(bq, np.uint32), _c(bk, np.uint32)
+    muq, muk = _c(muq, np.float64), _c(muk, np.float64)
+    vq, sv = _c(vq, np.int8), _c(sv, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    N = bq.shape[1]
+    R = row_hi - row_lo
+    out = np.zeros((R, d), np.float64)
+    pq = np.zeros((R, N), np.uint8) if want_pq else None
+    l = np.zeros(R, np.float64)
+    m = np.zeros(R, np.float64)
+    _load().bao_attention_rows(_ptr(bq), _ptr(muq), _ptr(bk), _ptr(muk), _ptr(vq), _ptr(sv),
+                               bias_kind, _ptr(b), ld, gh, gw, H, N, d, bh, row_lo, row_hi,
+                               _ptr(out), _ptr(pq), _ptr(l), _ptr(m))
+    return out, pq, l, m
+
+
+def attention_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, B, H, d, nthreads=0):
+    """Full forward, out [BH, N, d] float64; returns (out, threads_used)."""
+    bq, bk = _c(bq, np.uint32), _c(bk, np.uint32)
+    muq, muk = _c(muq, np.float64), _c(muk, np.float64)
+    vq, sv = _c(vq, np.int8), _c(sv, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    N = bq.shape[1]
+    out = np.zeros((B * H, N, d), np.float64)
+    used = _load().bao_attention_fwd(_ptr(bq), _ptr(muq), _ptr(bk), _ptr(muk), _ptr(vq), _ptr(sv),
+                                     bias_kind, _ptr(b), ld, gh, gw, B, H, N, d, _ptr(out), nthreads)
+    return out, used
+
+
+def forward(q, k, v, bias_kind=BIAS_NONE, bias=None, ld=0, gh=0, gw=0, nthreads=0):
+    """Whole pipeline from raw q, k, v [B, H, N, d] (float32 values).
+
+    Returns a dict with every intermediate the tests compare: bits_q, mu_q,
+    bits_k, mu_k (shaped [BH, N, ...]), vq [BH, N, d], sv [BH, d] and
+    out [B, H, N, d] float64.
+    """
+    B, H, N, d = q.shape
+    bq, muq = pack(np.asarray(q, np.float32).reshape(B * H, N, d))
+    bk, muk = pack(np.asarray(k, np.float32).reshape(B * H, N, d))
+    vq, sv = quant_v(np.asarray(v, np.float32).reshape(B * H, N, d))
+    out, used = attention_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, B, H, d, nthreads)
+    return dict(bits_q=bq, mu_q=muq, bits_k=bk, mu_k=muk, vq=vq, sv=sv,
+                out=out.reshape(B, H, N, d), threads=used)

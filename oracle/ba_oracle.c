@@ -1,0 +1,278 @@
+/*
+ * ba_oracle.c -- plain CPU oracle for the BinaryAttention forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library under bit_qk_attention_ba_b200/) never calls it, and this
+ * file shares no code, header, table or helper with that path.
+ *
+ * Source cited throughout ("BA notes"): the paper-notes page
+ *   "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+ *    Transformers" (CVPR 2026, arXiv 2603.09582),
+ * sections "Key design 1: Scaled Binary Representations" (KD1),
+ * "Key design 2: Bias Enhancement" (KD2), "Key design 3: Hybrid
+ * Quantization" (KD3) and "Overall framework" (FA2 tiled attention).
+ *
+ * Everything is written for clarity, not speed: straight loops, double
+ * precision, exact row maximum, int64 sums.  The only decisions taken in a
+ * lower precision are the ones that produce integers the CUDA path must match
+ * bit for bit (the int8 V codes): those are taken in IEEE fp32, the precision
+ * of the kernel, as the parity rules require.
+ *
+ * Readings where the page is silent (each also listed in the design notes):
+ *   - sign(x) is +1 when x >= 0 (so -0.0 -> +1) and -1 otherwise; NaN -> -1.
+ *   - mu is one scale per token: mean |x| over the d channels.  This is the
+ *     closed-form minimiser of || x - mu * sign(x) ||^2.
+ *   - sqrt(d) uses the true head dimension d, never the padded width.
+ *   - P~ = exp(S - m) with m the exact row maximum; pq = round-half-even(255 P~);
+ *     the row denominator l is the sum of the UNQUANTISED P~.
+ *   - V is quantised per (batch, head, channel) over the N tokens: symmetric
+ *     absmax / 127, IEEE fp32 division, round-half-even, clamp to [-127, 127];
+ *     an all-zero channel gets scale 0 and codes 0.
+ *   - The bias is shared over the batch.  Dense: b[h][i][j] at row stride ld.
+ *     2-D relative position: token i sits at (i / gw, i % gw); the table index
+ *     is (ri - rj + gh - 1) * (2 gw - 1) + (ci - cj + gw - 1).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* Number of 32-bit words that hold d sign bits. */
+int bao_words(int d) { return (d + 31) / 32; }
+
+/* KD1: sign of one value, as the +-1 integer the dot product uses. */
+static int sign_pm1(float x) { return (x >= 0.0f) ? +1 : -1; }
+
+/*
+ * KD1 (Scaled Binary Representations): sign-binarise each token and keep its
+ * magnitude as a per-token scale.
+ *   x    : [T, d] fp32 values (T = B*H*N tokens, channel fastest)
+ *   bits : [T, W] words, W = ceil(d/32); channel c -> word c/32, bit c%32
+ *          (least significant bit first); bit = 1 when sign is +1; unused
+ *          high bits of the last word are 0.
+ *   mu   : [T] mean |x| in double.
+ */
+void bao_pack(const float* x, int64_t T, int d, uint32_t* bits, double* mu)
+{
+    const int W = bao_words(d);
+    for (int64_t t = 0; t < T; ++t) {
+        const float* row = x + t * d;
+        for (int w = 0; w < W; ++w) {
+            uint32_t word = 0;
+            for (int b = 0; b < 32; ++b) {
+                int c = 32 * w + b;
+                if (c < d && sign_pm1(row[c]) == +1) word |= (1u << b);
+            }
+            bits[t * W + w] = word;
+        }
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) s += fabs((double)row[c]);
+        mu[t] = s / (double)d;
+    }
+}
+
+/* KD1, definition form: s.t over +-1 vectors taken straight from the values. */
+int32_t bao_dot_pm1(const float* q, const float* k, int d)
+{
+    int32_t z = 0;
+    for (int c = 0; c < d; ++c) z += sign_pm1(q[c]) * sign_pm1(k[c]);
+    return z;
+}
+
+/* Count set bits one at a time (no builtin, so it can be read by eye). */
+static int count_bits(uint32_t v)
+{
+    int n = 0;
+    for (int b = 0; b < 32; ++b) n += (int)((v >> b) & 1u);
+    return n;
+}
+
+/*
+ * KD1, XNOR/popcount form: s.t = d - 2 * hamming(bits_q, bits_k).  Padding
+ * bits are zero in both operands, so they add nothing to the Hamming distance.
+ */
+int32_t bao_dot_bits(const uint32_t* a, const uint32_t* b, int d)
+{
+    const int W = bao_words(d);
+    int ham = 0;
+    for (int w = 0; w < W; ++w) ham += count_bits(a[w] ^ b[w]);
+    return (int32_t)(d - 2 * ham);
+}
+
+/* Integer score matrix z[bh][i][j] = s_i . t_j for every (batch, head). */
+void bao_scores(const uint32_t* bq, const uint32_t* bk, int64_t BH, int N, int d,
+                int32_t* z)
+{
+    const int W = bao_words(d);
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < N; ++i)
+            for (int j = 0; j < N; ++j)
+                z[(bh * N + i) * (int64_t)N + j] =
+                    bao_dot_bits(bq + (bh * N + i) * W, bk + (bh * N + j) * W, d);
+}
+
+/* KD2 (Bias Enhancement): the additive bias b_ij of head h. */
+double bao_bias_value(int kind, const float* bias, int64_t ld, int h, int N,
+                      int gh, int gw, int i, int j)
+{
+    if (kind == 1) return (double)bias[((int64_t)h * N + i) * ld + j];
+    if (kind == 2) {
+        int ri = i / gw, ci = i % gw, rj = j / gw, cj = j % gw;
+        int64_t per_head = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+        int64_t idx = (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1);
+        return (double)bias[(int64_t)h * per_head + idx];
+    }
+    return 0.0;
+}
+
+/*
+ * KD3 (Hybrid Quantization), V side: channel-wise symmetric int8.
+ *   v  : [BH, N, d] fp32
+ *   vq : [BH, N, d] int8 codes (natural layout; the CUDA path's own layout is
+ *        its business, the tests rearrange)
+ *   sv : [BH, d] fp32 scales, sv = fl32(absmax / 127)
+ * The code of an element is round-half-even(fl32(v / sv)), clamped to +-127.
+ */
+void bao_quant_v(const float* v, int64_t BH, int N, int d, int8_t* vq, float* sv)
+{
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        for (int c = 0; c < d; ++c) {
+            float a = 0.0f;
+            for (int n = 0; n < N; ++n) {
+                float m = fabsf(v[(bh * N + n) * d + c]);
+                if (m > a) a = m;
+            }
+            volatile float s = a / 127.0f;   /* one IEEE fp32 division */
+            sv[bh * d + c] = s;
+            for (int n = 0; n < N; ++n) {
+                int q = 0;
+                if (s != 0.0f) {
+                    volatile float r = v[(bh * N + n) * d + c] / s;
+                    float rq = nearbyintf(r);  /* default mode: half to even */
+                    if (rq > 127.0f) rq = 127.0f;
+                    if (rq < -127.0f) rq = -127.0f;
+                    q = (int)rq;
+                }
+                vq[(bh * N + n) * d + c] = (int8_t)q;
+            }
+        }
+    }
+}
+
+/*
+ * The whole forward for query rows [row_lo, row_hi) of one (batch, head) bh:
+ *   S_ij  = muq_i * muk_j * (s_i . t_j) / sqrt(d) + b_ij          (KD2)
+ *   m_i   = max_j S_ij                                             (exact)
+ *   P~_ij = exp(S_ij - m_i),  l_i = sum_j P~_ij
+ *   pq_ij = round-half-even(255 * P~_ij)  in 0..255                (KD3)
+ *   O_ic  = sv_c * sum_j pq_ij * vq_jc / (255 * l_i)               (KD3)
+ * Inputs use the layouts above (bits [BH,N,W], mu [BH,N], vq [BH,N,d],
+ * sv [BH,d]).  out receives (row_hi - row_lo) rows of d doubles.  pq_out,
+ * l_out and m_out are optional (NULL to skip) and receive the same rows.
+ */
+void bao_attention_rows(const uint32_t* bq, const double* muq,
+                        const uint32_t* bk, const double* muk,
+                        const int8_t* vq, const float* sv,
+                        int bias_kind, const float* bias, int64_t ld, int gh, int gw,
+                        int H, int N, int d, int64_t bh, int row_lo, int row_hi,
+                        double* out, uint8_t* pq_out, double* l_out, double* m_out)
+{
+    const int W = bao_words(d);
+    const int h = (int)(bh % H);
+    const double rsd = sqrt((double)d);
+    double* S = (double*)malloc(sizeof(double) * (size_t)N);
+    int* pq = (int*)malloc(sizeof(int) * (size_t)N);
+
+    for (int i = row_lo; i < row_hi; ++i) {
+        const uint32_t* qi = bq + (bh * N + i) * W;
+        for (int j = 0; j < N; ++j) {
+            int32_t z = bao_dot_bits(qi, bk + (bh * N + j) * W, d);
+            S[j] = muq[bh * N + i] * muk[bh * N + j] * (double)z / rsd
+                 + bao_bias_value(bias_kind, bias, ld, h, N, gh, gw, i, j);
+        }
+        double m = S[0];
+        for (int j = 1; j < N; ++j) if (S[j] > m) m = S[j];
+        double l = 0.0;
+        for (int j = 0; j < N; ++j) {
+            double p = exp(S[j] - m);
+            l += p;
+            pq[j] = (int)nearbyint(255.0 * p);
+        }
+        int r = i - row_lo;
+        for (int c = 0; c < d; ++c) {
+            int64_t acc = 0;
+            for (int j = 0; j < N; ++j) acc += (int64_t)pq[j] * vq[(bh * N + j) * d + c];
+            out[(int64_t)r * d + c] = (double)sv[bh * d + c] * (double)acc / (255.0 * l);
+        }
+        if (pq_out) for (int j = 0; j < N; ++j) pq_out[(int64_t)r * N + j] = (uint8_t)pq[j];
+        if (l_out) l_out[r] = l;
+        if (m_out) m_out[r] = m;
+    }
+    free(S);
+    free(pq);
+}
+
+/* ---- threaded driver over independent (batch, head, row-block) units ---- */
+
+typedef struct {
+    const uint32_t* bq; const double* muq; const uint32_t* bk; const double* muk;
+    const int8_t* vq; const float* sv;
+    int bias_kind; const float* bias; int64_t ld; int gh, gw;
+    int H, N, d; int64_t BH;
+    double* out;
+    int64_t n_units; int rows_per_unit;
+    int64_t next;                 /* next unit to take, guarded by lock */
+    pthread_mutex_t lock;
+} fwd_job;
+
+static void* fwd_worker(void* arg)
+{
+    fwd_job* J = (fwd_job*)arg;
+    int blocks = (J->N + J->rows_per_unit - 1) / J->rows_per_unit;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t u = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= J->n_units) break;
+        int64_t bh = u / blocks;
+        int lo = (int)(u % blocks) * J->rows_per_unit;
+        int hi = lo + J->rows_per_unit < J->N ? lo + J->rows_per_unit : J->N;
+        bao_attention_rows(J->bq, J->muq, J->bk, J->muk, J->vq, J->sv,
+                           J->bias_kind, J->bias, J->ld, J->gh, J->gw,
+                           J->H, J->N, J->d, bh, lo, hi,
+                           J->out + (bh * J->N + lo) * J->d, NULL, NULL, NULL);
+    }
+    return NULL;
+}
+
+/*
+ * Full forward over all B*H heads, out [BH, N, d] doubles.  nthreads <= 0
+ * uses every online core.  Returns the number of threads used.
+ */
+int bao_attention_fwd(const uint32_t* bq, const double* muq,
+                      const uint32_t* bk, const double* muk,
+                      const int8_t* vq, const float* sv,
+                      int bias_kind, const float* bias, int64_t ld, int gh, int gw,
+                      int B, int H, int N, int d, double* out, int nthreads)
+{
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    fwd_job J;
+    memset(&J, 0, sizeof(J));
+    J.bq = bq; J.muq = muq; J.bk = bk; J.muk = muk; J.vq = vq; J.sv = sv;
+    J.bias_kind = bias_kind; J.bias = bias; J.ld = ld; J.gh = gh; J.gw = gw;
+    J.H = H; J.N = N; J.d = d; J.BH = (int64_t)B * H; J.out = out;
+    J.rows_per_unit = 16;
+    J.n_units = J.BH * ((N + J.rows_per_unit - 1) / J.rows_per_unit);
+    J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, fwd_worker, &J);
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return nthreads;
+}
