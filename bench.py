@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the BinaryAttention forward hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input already in
+HBM: pack Q, pack K (sign bits + per-token scale), quantise V (channel-wise
+int8), fused attention (binary QK, bias, online softmax, u8 P, integer PV).
+Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Metric: effective TOPS = 4*B*H*N^2*d per step / step time (higher is better);
+ms_per_step and the fused kernel's roofline fraction are reported alongside.
+Multi-GPU (torchrun): every rank runs its own copy of the workload (the (b, h)
+units are independent, no collective on the data path); value = all ranks'
+operations / max-over-ranks time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_qk_attention_ba_b200.workloads import BIAS_KIND, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "binary attention effective TOPS (4*B*H*N^2*d per step)"
+L2_BYTES = 126 * 2 ** 20
+ATTN_SRC = os.path.join(ROOT, "bit_qk_attention_ba_b200", "csrc", "ba_attn_tc.cu")
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    """Measured B200 peaks (generated file), else the recipe's fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def attn_bytes(w, out_bytes):
+    """Algorithmic bytes of one attention call: packed Q and K bits, both
+    scales, int8 V, V scales, the bias (read once, shared over the batch), and
+    the output."""
+    BH, N, d = w.B * w.H, w.N, w.d
+    W = (d + 31) // 32
+    b = 2 * BH * N * W * 4 + 2 * BH * N * 4 + BH * N * d + BH * d * 4 + BH * N * d * out_bytes
+    if w.bias == "dense":
+        b += w.H * N * N * 4
+    elif w.bias == "relpos2d":
+        gh, gw = w.grid
+        b += w.H * (2 * gh - 1) * (2 * gw - 1) * 4
+    return b
+
+
+def source_hash(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_tag, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel_tag, workload))
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != source_hash(ATTN_SRC):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def smi_id(dev):
+    """nvidia-smi -i selector for a torch device (its UUID when available)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x for x in vis.split(",") if x.strip()]
+    return ids[dev.index].strip() if dev.index < len(ids) else str(dev.index)
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a float over ranks (identity for one process)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, w, rank, local_rank, world):
+    import torch
+    import bit_qk_attention_ba_b200 as ba
+    from bit_qk_attention_ba_b200 import _native as NAT
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    inp = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {n: torch.from_numpy(inp[n]).to(tdt).pin_memory() for n in ("q", "k", "v")}
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
+    host_bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).pin_memory()
+    kind, ld, grid = BIAS_KIND[w.bias], inp["ld"], w.grid
+    out_dtype = tdt
+    out_bytes = 2 if out_dtype == torch.bfloat16 else 4
+    d = w.d
+    bq, muq = ba.pack_qk(q)
+    bk, muk = ba.pack_qk(k)
+    vq, sv = ba.quant_v(v)
+    out = torch.empty((w.B, w.H, w.N, d), dtype=out_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + (bias.numel() * 4 if bias is not None else 0)
+    flush = None
+    if in_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        ba.pack_qk(q, bq, muq)
+        ba.pack_qk(k, bk, muk)
+        ba.quant_v(v, vq, sv)
+        if i is not None:
+            a0[i].record(stream)
+        ba.attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=bias, bias_kind=kind, ld=ld, grid=grid,
+                         out=out, variant=args.variant)
+        if i is not None:
+            a1[i].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ba.check_device_status(dev) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(smi_id(dev)) as clk:
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record(stream)
+            step(i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    attn_ms = [x.elapsed_time(y) for x, y in zip(a0, a1)]
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(total_ms, world, dev)
+    status = ba.check_device_status(dev)
+    clocks = clk.summary()
+
+    # end to end through the public API: pinned host inputs -> device -> host output
+    host_out = torch.empty((w.B, w.H, w.N, d), dtype=out_dtype).pin_memory()
+    e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bd = torch.empty_like(bias) if bias is not None else None
+
+    def e2e_step():
+        qd.copy_(host["q"], non_blocking=True)
+        kd.copy_(host["k"], non_blocking=True)
+        vd.copy_(host["v"], non_blocking=True)
+        if bd is not None:
+            bd.copy_(host_bias, non_blocking=True)
+        o = ba.forward(qd, kd, vd, bias=bd, bias_kind=kind, ld=ld, grid=grid, out_dtype=out_dtype,
+                       variant=args.variant)
+        host_out.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+    h2d = in_bytes
+    d2h = host_out.numel() * host_out.element_size()
+
+    ms = total_ms / args.steps
+    ops = w.ops
+    value = world * ops / (ms * 1e-3) / 1e12
+    pk = peaks()
+    attn_t = statistics.median(attn_ms) * 1e-3
+    int8_peak = (pk["bf16_sus"]) * 2.0          # int8 dense = 2x bf16 dense (nominal ratio)
+    abytes = attn_bytes(w, out_bytes)
+    t_tensor, t_hbm = ops / (int8_peak * 1e12), abytes / (pk["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": ops / attn_t / 1e12, "peak": int8_peak, "unit": "TOPS"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / attn_t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic("attn_tc", w.name)
+    roof["kernel_us"] = attn_t * 1e6
+    roof["peak_source"] = ("int8 = 2 x measured sustained bf16 (%s)" % pk["src"]) if roof["bound"] == "tensor" \
+        else "measured HBM copy (%s)" % pk["src"]
+    roof["algorithmic_bytes"] = abytes
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8/s8/b1 (QK b1, PV u8xs8->s32, softmax fp32)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
+                   "bias": w.bias, "parallelism": "replicas%d" % world,
+                   "l2": "flushed between steps" if flush is not None else "inputs larger than L2",
+                   "qk_variant": args.variant},
+        "roofline": roof,
+        "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return line
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_baseline(w, inp, budget_s=15.0, heads=1):
+    """Time the oracle as it stands on a bounded sample of this workload:
+    pack/quantise the first `heads` heads, then the full forward of a block of
+    query rows of those heads (every key), and scale to the whole workload."""
+    import oracle as O
+    O.build()
+    d, N = w.d, w.N
+    gh, gw = w.grid
+    kind = BIAS_KIND[w.bias]
+    q = inp["q"].reshape(-1, N, d)[:heads]
+    k = inp["k"].reshape(-1, N, d)[:heads]
+    v = inp["v"].reshape(-1, N, d)[:heads]
+    t0 = time.perf_counter()
+    bq, muq = O.pack(q)
+    bk, muk = O.pack(k)
+    vq, sv = O.quant_v(v)
+    t_pre = time.perf_counter() - t0
+    rows = min(N, 16)
+    t0 = time.perf_counter()
+    _, used = O.attention_fwd_rows(bq, muq, bk, muk, vq, sv, kind, inp["bias"], inp["ld"], gh, gw,
+                                   heads, w.H, d, 0, rows)
+    t_probe = time.perf_counter() - t0
+    target = max(rows, min(N, int(rows * budget_s / max(t_probe, 1e-6))))
+    t0 = time.perf_counter()
+    _, used = O.attention_fwd_rows(bq, muq, bk, muk, vq, sv, kind, inp["bias"], inp["ld"], gh, gw,
+                                   heads, w.H, d, 0, target)
+    t_attn = time.perf_counter() - t0
+    BH = w.B * w.H
+    t_full = t_pre * BH / heads + t_attn * (BH * N) / (heads * target)
+    return {"value": w.ops / t_full / 1e12, "unit": "TOPS", "cores": used, "kind": "oracle",
+            "sample": "%d head(s) x %d of %d query rows (all keys) + pre-passes of those heads, "
+                      "%.1f s wall, scaled to the full workload" % (heads, target, N, t_pre + t_attn),
+            "seconds_full_workload_est": t_full}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return None
+    inp = make_inputs(w)
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, inp, budget_s=per_step)
+        if i >= args.warmup:
+            vals.append(cb)
+    value = statistics.median(c["value"] for c in vals)
+    ms = w.ops / (value * 1e12) * 1e3
+    cb = dict(vals[-1])
+    cb["value"] = value
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
+                   "bias": w.bias, "parallelism": "cpu oracle"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="hires16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 3 tcgen05 i8, 4 tcgen05 f8")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, local_rank, world = dist_env()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+    else:
+        line = run_ours(args, w, rank, local_rank, world)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+"""B200-native BinaryAttention forward (sm_100a CUDA behind a C ABI).
+
+Python surface over libba (include/ba.h).  Tensors are torch CUDA tensors;
+the functions allocate outputs with torch (the library itself allocates
+nothing) and queue work on torch's current stream.
+
+Method: the paper-notes page "BinaryAttention: One-Bit QK-Attention for Vision
+and Diffusion Transformers" (CVPR 2026): Key design 1 (sign Q/K with per-token
+scales, XNOR/popcount scores), Key design 2 (additive bias), Key design 3 (u8
+P with scale 1/255, channel-wise int8 V, integer PV).
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _native as N
+
+__all__ = ["pack_qk", "quant_v", "attention_fwd", "scores_debug", "forward", "check_device_status",
+           "words", "vq_ld"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return N.BA_BF16
+    if t.dtype == torch.float32:
+        return N.BA_F32
+    raise TypeError("expected float32 or bfloat16, got %s" % t.dtype)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def words(d: int) -> int:
+    return (d + 31) // 32
+
+
+def vq_ld(n: int) -> int:
+    return (n + 15) // 16 * 16
+
+
+def pack_qk(x, bits=None, mu=None):
+    """Sign bits [B,H,N,W] (int32 storage of the uint32 words) and mu [B,H,N]."""
+    torch = _torch()
+    _need_cuda(x)
+    B, H, Nn, d = x.shape
+    if bits is None:
+        bits = torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=x.device)
+    if mu is None:
+        mu = torch.empty((B, H, Nn), dtype=torch.float32, device=x.device)
+    N.call("ba_pack_qk", _p(x), _dt(x), B, H, Nn, d, _p(bits), _p(mu), _stream(x.device))
+    return bits, mu
+
+
+def quant_v(v, vq=None, sv=None):
+    """int8 codes [B,H,d,ldv] (channel-major) and scales sv [B,H,d]."""
+    torch = _torch()
+    _need_cuda(v)
+    B, H, Nn, d = v.shape
+    if vq is None:
+        vq = torch.empty((B, H, d, vq_ld(Nn)), dtype=torch.int8, device=v.device)
+    if sv is None:
+        sv = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
+    N.call("ba_quant_v", _p(v), _dt(v), B, H, Nn, d, _p(vq), _p(sv), _stream(v.device))
+    return vq, sv
+
+
+def _bias_args(bias, bias_kind, ld, grid):
+    if bias is None or bias_kind == N.BA_BIAS_NONE:
+        return N.BA_BIAS_NONE, None, 0, 0, 0
+    _need_cuda(bias)
+    gh, gw = grid if grid else (0, 0)
+    if bias_kind == N.BA_BIAS_DENSE and not ld:
+        ld = bias.shape[-1]
+    return bias_kind, _p(bias), int(ld or 0), int(gh), int(gw)
+
+
+def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None,
+                  out=None, out_dtype=None, variant=N.BA_QK_AUTO):
+    """Fused forward; returns out [B,H,N,d] (float32 unless out_dtype given)."""
+    torch = _torch()
+    _need_cuda(bq, muq, bk, muk, vq, sv)
+    B, H, Nn = muq.shape
+    if out is None:
+        out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=muq.device)
+    kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
+    N.call("ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
+           B, H, Nn, d, _p(out), _dt(out), int(variant), _stream(muq.device))
+    return out
+
+
+def scores_debug(bq, bk, d, z=None):
+    """Integer binary scores z [B,H,N,N] int32."""
+    torch = _torch()
+    _need_cuda(bq, bk)
+    B, H, Nn, _ = bq.shape
+    if z is None:
+        z = torch.empty((B, H, Nn, Nn), dtype=torch.int32, device=bq.device)
+    N.call("ba_scores_debug", _p(bq), _p(bk), B, H, Nn, d, _p(z), _stream(bq.device))
+    return z
+
+
+def forward(q, k, v, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None, out_dtype=None,
+            variant=N.BA_QK_AUTO):
+    """The whole hot path: pack Q, pack K, quantise V, fused attention."""
+    d = q.shape[-1]
+    bq, muq = pack_qk(q)
+    bk, muk = pack_qk(k)
+    vq, sv = quant_v(v)
+    return attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=bias, bias_kind=bias_kind, ld=ld, grid=grid,
+                         out_dtype=out_dtype or q.dtype, variant=variant)
+
+
+def check_device_status(device=None) -> int:
+    """Synchronise and return the device status word (0 = no kernel failure)."""
+    code = ctypes.c_int(0)
+    st = N.lib().ba_check_device_status(_stream(device), ctypes.byref(code))
+    if st not in (N.BA_OK, N.BA_ERR_DEVICE_STATUS):
+        N.check("ba_check_device_status", st)
+    return code.value

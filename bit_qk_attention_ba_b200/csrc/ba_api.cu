@@ -1,0 +1,200 @@
+// ba_api.cu -- the C ABI of libba: argument checks, dispatch, status word.
+//
+// Every entry point validates its arguments on the host before queueing any
+// work, launches asynchronously on the caller's stream and returns a status
+// code; nothing throws across the ABI and nothing is allocated.
+#include <mutex>
+
+#include "ba_common.cuh"
+
+namespace ba {
+
+cudaError_t launch_pack(const void* x, ba_dtype dt, int64_t tokens, int d, uint32_t* bits,
+                        float* mu, cudaStream_t st, int sm_count);
+cudaError_t launch_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int8_t* vq,
+                           float* sv, cudaStream_t st);
+cudaError_t launch_scores(const uint32_t* bq, const uint32_t* bk, int B, int H, int N, int d,
+                          int32_t* z, cudaStream_t st);
+cudaError_t launch_attn_simt(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                             const int8_t* vq, const float* sv, int bias_kind, const float* bias,
+                             int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                             void* out, ba_dtype out_dt, cudaStream_t st);
+// Returns cudaErrorNotSupported when the tensor-core path cannot take the shape.
+cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv, int bias_kind, const float* bias,
+                           int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                           void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st);
+bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d);
+
+// One status word per device; kernels OR failure bits into it.
+__device__ unsigned g_device_status;
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+int current_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+// Per-device set-up, done once with the device current.
+bool device_setup(int dev)
+{
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_status_ptr[dev]) return true;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return false;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    g_sm_count[dev] = sms;
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+    return true;
+}
+}  // namespace
+
+unsigned* device_status_ptr()
+{
+    const int dev = current_device();
+    return device_setup(dev) ? g_status_ptr[dev] : nullptr;
+}
+
+static int sm_count()
+{
+    const int dev = current_device();
+    return device_setup(dev) ? g_sm_count[dev] : 0;
+}
+
+static bool sizes_ok(int B, int H, int N, int d)
+{
+    return B >= 1 && H >= 1 && N >= 1 && d >= 1 && d <= 128 && (int64_t)B * H <= 65535 &&
+           (int64_t)N <= (1 << 24);
+}
+
+static bool ptr_ok(const void* p) { return p != nullptr && aligned(p, 16); }
+
+static ba_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BA_OK : BA_ERR_CUDA; }
+
+static bool bias_ok(int kind, const float* bias, int64_t ld, int gh, int gw, int N)
+{
+    if (kind == BA_BIAS_NONE) return true;
+    if (kind == BA_BIAS_DENSE) return ptr_ok(bias) && ld >= N && ld % 4 == 0;
+    if (kind == BA_BIAS_RELPOS2D)
+        return ptr_ok(bias) && gh >= 1 && gw >= 1 && (int64_t)gh * gw == N;
+    return false;
+}
+
+}  // namespace ba
+
+using namespace ba;
+
+extern "C" {
+
+int ba_words(int d) { return words_for(d); }
+
+int64_t ba_vq_ld(int N) { return round_up64(N, 16); }
+
+const char* ba_status_string(ba_status s)
+{
+    switch (s) {
+        case BA_OK: return "BA_OK";
+        case BA_ERR_INVALID_ARG: return "BA_ERR_INVALID_ARG";
+        case BA_ERR_UNSUPPORTED: return "BA_ERR_UNSUPPORTED";
+        case BA_ERR_CUDA: return "BA_ERR_CUDA";
+        case BA_ERR_DEVICE_STATUS: return "BA_ERR_DEVICE_STATUS";
+    }
+    return "BA_ERR_UNKNOWN";
+}
+
+ba_status ba_pack_qk(const void* x, ba_dtype dt, int B, int H, int N, int d,
+                     uint32_t* bits, float* mu, void* stream)
+{
+    if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(x) || !ptr_ok(bits) || !ptr_ok(mu)) return BA_ERR_INVALID_ARG;
+    const int sms = sm_count();
+    if (sms <= 0) return BA_ERR_CUDA;
+    return from_cuda(launch_pack(x, dt, (int64_t)B * H * N, d, bits, mu,
+                                 static_cast<cudaStream_t>(stream), sms));
+}
+
+ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
+                     int8_t* vq, float* sv, void* stream)
+{
+    if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(v) || !ptr_ok(vq) || !ptr_ok(sv)) return BA_ERR_INVALID_ARG;
+    return from_cuda(launch_quant_v(v, dt, B, H, N, d, vq, sv, static_cast<cudaStream_t>(stream)));
+}
+
+ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, int N, int d,
+                          int32_t* z, void* stream)
+{
+    if (!sizes_ok(B, H, N, d)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq) || !ptr_ok(bk) || !ptr_ok(z)) return BA_ERR_INVALID_ARG;
+    if (ceil_div(N, 64) > 65535) return BA_ERR_UNSUPPORTED;
+    return from_cuda(launch_scores(bq, bk, B, H, N, d, z, static_cast<cudaStream_t>(stream)));
+}
+
+ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
+                                   const uint32_t* bk, const float* muk,
+                                   const int8_t* vq, const float* sv,
+                                   int bias_kind, const float* bias, int64_t bias_ld,
+                                   int grid_h, int grid_w,
+                                   int B, int H, int N, int d,
+                                   void* out, ba_dtype out_dt, int variant, void* stream)
+{
+    if (!sizes_ok(B, H, N, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq) || !ptr_ok(muq) || !ptr_ok(bk) || !ptr_ok(muk) || !ptr_ok(vq) || !ptr_ok(sv) ||
+        !ptr_ok(out))
+        return BA_ERR_INVALID_ARG;
+    if (!bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N)) return BA_ERR_INVALID_ARG;
+    if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_TC_I8 && variant != BA_QK_TC_F8)
+        return BA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (variant == BA_QK_POPC)
+        return from_cuda(launch_attn_simt(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
+                                          grid_w, B, H, N, d, out, out_dt, st));
+    const bool tc_ok = attn_tc_supports(bias_kind, grid_h, grid_w, N, d);
+    if (!tc_ok) {
+        if (variant != BA_QK_AUTO) return BA_ERR_UNSUPPORTED;
+        return from_cuda(launch_attn_simt(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
+                                          grid_w, B, H, N, d, out, out_dt, st));
+    }
+    unsigned* status = device_status_ptr();
+    if (!status) return BA_ERR_CUDA;
+    const cudaError_t e = launch_attn_tc(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
+                                         B, H, N, d, out, out_dt, variant, status, st);
+    if (e == cudaErrorNotSupported) return BA_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
+                           const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv,
+                           int bias_kind, const float* bias, int64_t bias_ld,
+                           int grid_h, int grid_w,
+                           int B, int H, int N, int d,
+                           void* out, ba_dtype out_dt, void* stream)
+{
+    return ba_attention_fwd_variant(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
+                                    B, H, N, d, out, out_dt, BA_QK_AUTO, stream);
+}
+
+ba_status ba_check_device_status(void* stream, int* code)
+{
+    unsigned* p = device_status_ptr();
+    if (!p) return BA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned host = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BA_ERR_CUDA;
+    if (cudaMemcpy(&host, p, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return BA_ERR_CUDA;
+    if (host != 0 && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return BA_ERR_CUDA;
+    if (code) *code = (int)host;
+    return host ? BA_ERR_DEVICE_STATUS : BA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+/*
+ * ba.h -- C ABI of libba, the B200 (sm_100a) BinaryAttention forward pass.
+ *
+ * Method source ("BA notes"): the paper-notes page "BinaryAttention: One-Bit
+ * QK-Attention for Vision and Diffusion Transformers" (CVPR 2026, arXiv
+ * 2603.09582).  Sections cited below:
+ *   KD1  Key design 1, Scaled Binary Representations (sign Q/K + scale mu,
+ *        XNOR/popcount dot product)
+ *   KD2  Key design 2, Bias Enhancement (S = mu_q mu_k s.t / sqrt(d) + b)
+ *   KD3  Key design 3, Hybrid Quantization (P as u8 with scale 1/255, V as
+ *        channel-wise int8, integer PV product)
+ *   FW   Overall framework (tiled attention in the FlashAttention2 style)
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *     in the layout stated, and 16-byte aligned.  The library allocates no
+ *     device memory and never synchronises: work is queued on `stream` (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Arguments are validated before anything is queued; an invalid call
+ *     returns BA_ERR_INVALID_ARG (or BA_ERR_UNSUPPORTED) and queues nothing.
+ *   - A launch failure reported by the CUDA runtime returns BA_ERR_CUDA.
+ *   - Kernels that wait on hardware barriers give up after a bounded number of
+ *     polls, record a code in a device status word and exit cleanly;
+ *     ba_check_device_status() reports it (BA_ERR_DEVICE_STATUS).
+ *   - Sizes: B, H, N >= 1; 1 <= d <= 128.  Tokens are [B, H, N] in that order.
+ *   - Nothing throws across the ABI.
+ */
+#ifndef BA_H_
+#define BA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BA_OK = 0,
+    BA_ERR_INVALID_ARG = 1,    /* bad size, null or misaligned pointer */
+    BA_ERR_UNSUPPORTED = 2,    /* valid request this build cannot serve */
+    BA_ERR_CUDA = 3,           /* the CUDA runtime reported an error */
+    BA_ERR_DEVICE_STATUS = 4   /* a kernel recorded a failure (see below) */
+} ba_status;
+
+typedef enum { BA_F32 = 0, BA_BF16 = 1 } ba_dtype;
+
+/* KD2: which additive bias b_ij enters the scores. */
+typedef enum {
+    BA_BIAS_NONE = 0,
+    BA_BIAS_DENSE = 1,     /* fp32 [H, N, ld], b_ij = bias[h][i][j]; ld >= N, ld % 4 == 0 */
+    BA_BIAS_RELPOS2D = 2   /* fp32 [H, (2 gh - 1) * (2 gw - 1)], N == gh * gw, see below */
+} ba_bias_kind;
+
+/* How the binary Q.K contraction runs inside ba_attention_fwd_variant. */
+typedef enum {
+    BA_QK_AUTO = 0,        /* the fastest path this build has for the shape */
+    BA_QK_POPC = 1,        /* CUDA cores: XOR + popcount on 32-bit words */
+    BA_QK_TC_I8 = 3,       /* tcgen05 kind::i8, +-1 int8 operands, s32 in TMEM */
+    BA_QK_TC_F8 = 4        /* tcgen05 kind::f8f6f4, +-1 e4m3 operands, f32 in TMEM */
+} ba_qk_variant;
+
+/* Number of 32-bit words per token in the packed sign layout: ceil(d / 32). */
+int ba_words(int d);
+
+/* Row stride (bytes = int8 elements) of the int8 V layout: N rounded up to 16. */
+int64_t ba_vq_ld(int N);
+
+/*
+ * KD1 -- sign-binarise Q or K and take the per-token scale.
+ *   x    : [B, H, N, d] values, dtype dt (BA_F32 or BA_BF16)
+ *   bits : [B, H, N, W] uint32, W = ba_words(d).  Channel c is bit c % 32 of
+ *          word c / 32 (least significant bit first); the bit is 1 when
+ *          x >= 0 (so -0.0 gives 1, NaN gives 0).  Unused high bits are 0.
+ *   mu   : [B, H, N] fp32, mu = (sum_c |x_c|) / d, the scale that minimises
+ *          || x - mu sign(x) ||^2 (one scale per token; the page says only
+ *          that mu keeps the token's magnitude).
+ */
+ba_status ba_pack_qk(const void* x, ba_dtype dt, int B, int H, int N, int d,
+                     uint32_t* bits, float* mu, void* stream);
+
+/*
+ * KD3 -- channel-wise int8 quantisation of V.
+ *   v  : [B, H, N, d] values, dtype dt
+ *   vq : [B, H, d, ldv] int8 with ldv = ba_vq_ld(N): CHANNEL-major, keys
+ *        contiguous, so a tile of keys is a K-major operand of the PV product.
+ *        vq[b][h][c][j] = clamp(round_half_even(fl32(v_jc / sv_c)), -127, 127);
+ *        the columns j in [N, ldv) are written as 0.
+ *   sv : [B, H, d] fp32, sv_c = fl32(max_j |v_jc| / 127) (IEEE division); an
+ *        all-zero channel has sv = 0 and codes 0.
+ * Inputs must be finite.
+ */
+ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
+                     int8_t* vq, float* sv, void* stream);
+
+/*
+ * KD1-KD3 + FW -- the fused forward.  For every (b, h, i):
+ *   z_ij  = s_i . t_j = d - 2 popcount(bq_i XOR bk_j)                   (KD1)
+ *   S_ij  = muq_i muk_j z_ij / sqrt(d) + b_ij                            (KD2)
+ *   P~_ij = exp(S_ij - m_i) with m_i the running row maximum (FW),
+ *   pq_ij = round(255 P~_ij) in 0..255, l_i = sum_j P~_ij (unquantised)  (KD3)
+ *   O_ic  = sv_c * sum_j pq_ij vq_jc / (255 l_i)                         (KD3)
+ * Inputs: bq, bk [B, H, N, W] from ba_pack_qk; muq, muk [B, H, N];
+ *   vq [B, H, d, ldv] and sv [B, H, d] from ba_quant_v.
+ * Bias (shared over the batch): bias_kind selects none, dense or 2-D relative
+ *   position.  DENSE: bias_ld is the row stride in floats (>= N, multiple of
+ *   4).  RELPOS2D: token i sits at (i / grid_w, i % grid_w), N must equal
+ *   grid_h * grid_w, and b_ij = table[h][(ri - rj + grid_h - 1) *
+ *   (2 grid_w - 1) + (ci - cj + grid_w - 1)].
+ * out: [B, H, N, d] in out_dt (BA_F32 or BA_BF16).
+ * The running maximum means pq may differ from an exact-maximum quantisation
+ * by one unit; the result stays within the stated parity tolerance.
+ */
+ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
+                           const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv,
+                           int bias_kind, const float* bias, int64_t bias_ld,
+                           int grid_h, int grid_w,
+                           int B, int H, int N, int d,
+                           void* out, ba_dtype out_dt, void* stream);
+
+/* Same computation with an explicit QK contraction path (ba_qk_variant);
+ * BA_ERR_UNSUPPORTED if that path cannot serve the shape. */
+ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
+                                   const uint32_t* bk, const float* muk,
+                                   const int8_t* vq, const float* sv,
+                                   int bias_kind, const float* bias, int64_t bias_ld,
+                                   int grid_h, int grid_w,
+                                   int B, int H, int N, int d,
+                                   void* out, ba_dtype out_dt, int variant, void* stream);
+
+/*
+ * KD1 -- the integer binary score matrix, for checking and debugging.
+ *   z : [B, H, N, N] int32, z[b][h][i][j] = d - 2 popcount(bq_i XOR bk_j).
+ */
+ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk,
+                          int B, int H, int N, int d, int32_t* z, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  BA_OK when no kernel recorded a failure, otherwise
+ * BA_ERR_DEVICE_STATUS with the recorded bits in *code (may be NULL).
+ */
+ba_status ba_check_device_status(void* stream, int* code);
+
+/* Static, human-readable name of a status code. */
+const char* ba_status_string(ba_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BA_H_ */

@@ -55,6 +55,8 @@ def _load():
     lib.bao_dot_bits.restype = ctypes.c_int32
     lib.bao_scores.argtypes = [P, P, i64, i32, i32, P]
     lib.bao_scores.restype = None
+    lib.bao_scores_rows.argtypes = [P, P, i32, i32, P, i32, P]
+    lib.bao_scores_rows.restype = None
     lib.bao_bias_value.argtypes = [i32, P, i64, i32, i32, i32, i32, i32, i32]
     lib.bao_bias_value.restype = ctypes.c_double
     lib.bao_quant_v.argtypes = [P, i64, i32, i32, P, P]
@@ -65,6 +67,9 @@ def _load():
     lib.bao_attention_fwd.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32,
                                       i32, i32, i32, i32, P, i32]
     lib.bao_attention_fwd.restype = i32
+    lib.bao_attention_fwd_rows.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32,
+                                           i64, i32, i32, i32, i32, i32, P, i32]
+    lib.bao_attention_fwd_rows.restype = i32
     _lib = lib
     return lib
 
@@ -112,6 +117,16 @@ def scores(bq, bk, d: int):
     return z
 
 
+def scores_rows(bq_head, bk_head, d: int, rows):
+    """z [len(rows), N] int32 for one head's bits [N, W] and chosen query rows."""
+    bq, bk = _c(bq_head, np.uint32), _c(bk_head, np.uint32)
+    r = _c(rows, np.int32)
+    N = bk.shape[0]
+    z = np.zeros((len(r), N), np.int32)
+    _load().bao_scores_rows(_ptr(bq), _ptr(bk), N, d, _ptr(r), len(r), _ptr(z))
+    return z
+
+
 def bias_value(kind, bias, ld, h, N, gh, gw, i, j) -> float:
     b = None if bias is None else _c(bias, np.float32)
     return float(_load().bao_bias_value(kind, _ptr(b), ld, h, N, gh, gw, i, j))
@@ -156,6 +171,21 @@ def attention_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, B, H, d
     out = np.zeros((B * H, N, d), np.float64)
     used = _load().bao_attention_fwd(_ptr(bq), _ptr(muq), _ptr(bk), _ptr(muk), _ptr(vq), _ptr(sv),
                                      bias_kind, _ptr(b), ld, gh, gw, B, H, N, d, _ptr(out), nthreads)
+    return out, used
+
+
+def attention_fwd_rows(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, n_heads, H, d,
+                       row_lo, row_hi, nthreads=0):
+    """Threaded rows [row_lo, row_hi) of heads [0, n_heads); out [n_heads, rows, d]."""
+    bq, bk = _c(bq, np.uint32), _c(bk, np.uint32)
+    muq, muk = _c(muq, np.float64), _c(muk, np.float64)
+    vq, sv = _c(vq, np.int8), _c(sv, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    N = bq.shape[1]
+    out = np.zeros((n_heads, row_hi - row_lo, d), np.float64)
+    used = _load().bao_attention_fwd_rows(_ptr(bq), _ptr(muq), _ptr(bk), _ptr(muk), _ptr(vq), _ptr(sv),
+                                          bias_kind, _ptr(b), ld, gh, gw, n_heads, H, N, d, row_lo, row_hi,
+                                          _ptr(out), nthreads)
     return out, used
 
 

@@ -114,6 +114,17 @@ void bao_scores(const uint32_t* bq, const uint32_t* bk, int64_t BH, int N, int d
                     bao_dot_bits(bq + (bh * N + i) * W, bk + (bh * N + j) * W, d);
 }
 
+/* The same for a block of rows: z[r][j] = s_(rows[r]) . t_j for one head,
+ * bq and bk pointing at that head's [N, W] bits. */
+void bao_scores_rows(const uint32_t* bq, const uint32_t* bk, int N, int d,
+                     const int32_t* rows, int n_rows, int32_t* z)
+{
+    const int W = bao_words(d);
+    for (int r = 0; r < n_rows; ++r)
+        for (int j = 0; j < N; ++j)
+            z[(int64_t)r * N + j] = bao_dot_bits(bq + (int64_t)rows[r] * W, bk + (int64_t)j * W, d);
+}
+
 /* KD2 (Bias Enhancement): the additive bias b_ij of head h. */
 double bao_bias_value(int kind, const float* bias, int64_t ld, int h, int N,
                       int gh, int gw, int i, int j)
@@ -223,6 +234,7 @@ typedef struct {
     int bias_kind; const float* bias; int64_t ld; int gh, gw;
     int H, N, d; int64_t BH;
     double* out;
+    int row_lo, row_hi;           /* query rows computed in every head */
     int64_t n_units; int rows_per_unit;
     int64_t next;                 /* next unit to take, guarded by lock */
     pthread_mutex_t lock;
@@ -231,32 +243,35 @@ typedef struct {
 static void* fwd_worker(void* arg)
 {
     fwd_job* J = (fwd_job*)arg;
-    int blocks = (J->N + J->rows_per_unit - 1) / J->rows_per_unit;
+    int span = J->row_hi - J->row_lo;
+    int blocks = (span + J->rows_per_unit - 1) / J->rows_per_unit;
     for (;;) {
         pthread_mutex_lock(&J->lock);
         int64_t u = J->next++;
         pthread_mutex_unlock(&J->lock);
         if (u >= J->n_units) break;
         int64_t bh = u / blocks;
-        int lo = (int)(u % blocks) * J->rows_per_unit;
-        int hi = lo + J->rows_per_unit < J->N ? lo + J->rows_per_unit : J->N;
+        int lo = J->row_lo + (int)(u % blocks) * J->rows_per_unit;
+        int hi = lo + J->rows_per_unit < J->row_hi ? lo + J->rows_per_unit : J->row_hi;
         bao_attention_rows(J->bq, J->muq, J->bk, J->muk, J->vq, J->sv,
                            J->bias_kind, J->bias, J->ld, J->gh, J->gw,
                            J->H, J->N, J->d, bh, lo, hi,
-                           J->out + (bh * J->N + lo) * J->d, NULL, NULL, NULL);
+                           J->out + (bh * span + (lo - J->row_lo)) * J->d, NULL, NULL, NULL);
     }
     return NULL;
 }
 
 /*
- * Full forward over all B*H heads, out [BH, N, d] doubles.  nthreads <= 0
- * uses every online core.  Returns the number of threads used.
+ * Threaded forward of query rows [row_lo, row_hi) in heads [0, n_heads):
+ * out [n_heads, row_hi - row_lo, d] doubles.  nthreads <= 0 uses every online
+ * core.  Returns the number of threads used.
  */
-int bao_attention_fwd(const uint32_t* bq, const double* muq,
-                      const uint32_t* bk, const double* muk,
-                      const int8_t* vq, const float* sv,
-                      int bias_kind, const float* bias, int64_t ld, int gh, int gw,
-                      int B, int H, int N, int d, double* out, int nthreads)
+int bao_attention_fwd_rows(const uint32_t* bq, const double* muq,
+                           const uint32_t* bk, const double* muk,
+                           const int8_t* vq, const float* sv,
+                           int bias_kind, const float* bias, int64_t ld, int gh, int gw,
+                           int64_t n_heads, int H, int N, int d, int row_lo, int row_hi,
+                           double* out, int nthreads)
 {
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
     if (nthreads < 1) nthreads = 1;
@@ -264,9 +279,10 @@ int bao_attention_fwd(const uint32_t* bq, const double* muq,
     memset(&J, 0, sizeof(J));
     J.bq = bq; J.muq = muq; J.bk = bk; J.muk = muk; J.vq = vq; J.sv = sv;
     J.bias_kind = bias_kind; J.bias = bias; J.ld = ld; J.gh = gh; J.gw = gw;
-    J.H = H; J.N = N; J.d = d; J.BH = (int64_t)B * H; J.out = out;
+    J.H = H; J.N = N; J.d = d; J.BH = n_heads; J.out = out;
+    J.row_lo = row_lo; J.row_hi = row_hi;
     J.rows_per_unit = 16;
-    J.n_units = J.BH * ((N + J.rows_per_unit - 1) / J.rows_per_unit);
+    J.n_units = J.BH * ((row_hi - row_lo + J.rows_per_unit - 1) / J.rows_per_unit);
     J.next = 0;
     pthread_mutex_init(&J.lock, NULL);
     pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
@@ -275,4 +291,15 @@ int bao_attention_fwd(const uint32_t* bq, const double* muq,
     free(th);
     pthread_mutex_destroy(&J.lock);
     return nthreads;
+}
+
+/* Full forward over all B*H heads, out [BH, N, d] doubles. */
+int bao_attention_fwd(const uint32_t* bq, const double* muq,
+                      const uint32_t* bk, const double* muk,
+                      const int8_t* vq, const float* sv,
+                      int bias_kind, const float* bias, int64_t ld, int gh, int gw,
+                      int B, int H, int N, int d, double* out, int nthreads)
+{
+    return bao_attention_fwd_rows(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw,
+                                  (int64_t)B * H, H, N, d, 0, N, out, nthreads);
 }

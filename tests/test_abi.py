@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls).
+
+The library must load, export every function include/ba.h declares, and
+reject invalid arguments before it touches the CUDA runtime.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_qk_attention_ba_b200 import build as B
+    B.build()
+    from bit_qk_attention_ba_b200 import _native
+    return _native.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ba_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("ba_pack_qk", "ba_quant_v", "ba_attention_fwd", "ba_scores_debug"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from bit_qk_attention_ba_b200 import _native
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in _native.SIGNATURES, "binding lacks " + name
+
+
+def test_pure_helpers(lib):
+    assert lib.ba_words(1) == 1 and lib.ba_words(32) == 1 and lib.ba_words(33) == 2
+    assert lib.ba_words(72) == 3 and lib.ba_words(128) == 4
+    assert lib.ba_vq_ld(1) == 16 and lib.ba_vq_ld(577) == 592 and lib.ba_vq_ld(16384) == 16384
+    assert lib.ba_status_string(0) == b"BA_OK"
+    assert lib.ba_status_string(1) == b"BA_ERR_INVALID_ARG"
+    assert lib.ba_status_string(4) == b"BA_ERR_DEVICE_STATUS"
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced (validation fails first)
+MIS = ctypes.c_void_p((1 << 20) + 4)      # misaligned
+
+
+@pytest.mark.parametrize("B,H,N,d", [(0, 1, 8, 64), (1, 0, 8, 64), (1, 1, 0, 64), (1, 1, 8, 0), (1, 1, 8, 129),
+                                     (70000, 1, 8, 64)])
+def test_bad_sizes_rejected(lib, B, H, N, d):
+    assert lib.ba_pack_qk(FAKE, 1, B, H, N, d, FAKE, FAKE, None) == 1
+    assert lib.ba_quant_v(FAKE, 1, B, H, N, d, FAKE, FAKE, None) == 1
+    assert lib.ba_scores_debug(FAKE, FAKE, B, H, N, d, FAKE, None) == 1
+    assert lib.ba_attention_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, 0, 0, 0,
+                                B, H, N, d, FAKE, 0, None) == 1
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    assert lib.ba_pack_qk(None, 1, 1, 1, 8, 64, FAKE, FAKE, None) == 1
+    assert lib.ba_pack_qk(MIS, 1, 1, 1, 8, 64, FAKE, FAKE, None) == 1
+    assert lib.ba_quant_v(FAKE, 1, 1, 1, 8, 64, MIS, FAKE, None) == 1
+    assert lib.ba_scores_debug(FAKE, None, 1, 1, 8, 64, FAKE, None) == 1
+    args = [FAKE] * 6
+    assert lib.ba_attention_fwd(*args[:5], None, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, MIS, 0, None) == 1
+
+
+def test_bad_dtypes_and_bias_rejected(lib):
+    assert lib.ba_pack_qk(FAKE, 7, 1, 1, 8, 64, FAKE, FAKE, None) == 1
+    args = [FAKE] * 6
+    # dense bias: ld < N, ld not a multiple of 4, null table
+    assert lib.ba_attention_fwd(*args, 1, FAKE, 4, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 1, FAKE, 9, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 1, None, 8, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    # rel-pos: N must equal grid_h * grid_w
+    assert lib.ba_attention_fwd(*args, 2, FAKE, 0, 3, 3, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 5, FAKE, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    # out dtype and unknown QK variant
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 9, None) == 1
+    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, 2, None) == 1
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle and has no CPU compute path."""
+    pkg = os.path.join(ROOT, "bit_qk_attention_ba_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "ba_oracle" not in text, f

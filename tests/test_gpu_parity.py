@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer outputs (sign bits, int8 V codes, binary scores) must match bit for
+bit.  Floating outputs: mu within fp32 summation error; the attention output
+within max-abs 2e-2 and mean-abs 2e-3 of the oracle (exact row max, fp64) on
+unit-scale V -- errors are divided by max(1, std of the value channel) so the
+x8 outlier channels of the DeiT-S workload get the same relative budget.  The
+GPU uses a running row max and fp32 arithmetic, so pq can move by one unit;
+that is what the tolerance covers.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from bit_qk_attention_ba_b200.workloads import BIAS_KIND, WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import bit_qk_attention_ba_b200 as ba  # noqa: E402
+from bit_qk_attention_ba_b200 import _native as NAT  # noqa: E402
+
+DEV = torch.device("cuda:0")
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+TC_VARIANTS = [NAT.BA_QK_TC_I8, NAT.BA_QK_TC_F8]
+
+
+def _gpu(x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(DEV).to(torch.bfloat16 if dtype == "bf16" else torch.float32).contiguous()
+
+
+def _bits(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def _vq_natural(vq_t, N):
+    """GPU layout [B,H,d,ldv] -> oracle layout [BH, N, d]."""
+    a = vq_t.cpu().numpy()
+    B, H, d, _ = a.shape
+    return np.ascontiguousarray(a[..., :N].transpose(0, 1, 3, 2)).reshape(B * H, N, d)
+
+
+def _assert_close(out_gpu, out_orc, v):
+    scale = np.maximum(1.0, v.astype(np.float64).std(axis=2, keepdims=True))
+    err = np.abs(out_gpu.astype(np.float64) - out_orc) / scale
+    assert np.isfinite(out_gpu).all()
+    assert err.max() <= MAX_ABS, "max-abs %.3g" % err.max()
+    assert err.mean() <= MEAN_ABS, "mean-abs %.3g" % err.mean()
+    return err
+
+
+def _bias_gpu(inp, w):
+    return None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(DEV)
+
+
+def _run_gpu(w, inp, variant=NAT.BA_QK_AUTO, out_dtype=torch.float32):
+    q, k, v = (_gpu(inp[n], w.dtype) for n in ("q", "k", "v"))
+    bq, muq = ba.pack_qk(q)
+    bk, muk = ba.pack_qk(k)
+    vq, sv = ba.quant_v(v)
+    out = ba.attention_fwd(bq, muq, bk, muk, vq, sv, w.d, bias=_bias_gpu(inp, w),
+                           bias_kind=BIAS_KIND[w.bias], ld=inp["ld"], grid=w.grid,
+                           out_dtype=out_dtype, variant=variant)
+    torch.cuda.synchronize()
+    return dict(bq=bq, muq=muq, bk=bk, muk=muk, vq=vq, sv=sv, out=out)
+
+
+def _oracle_full(w, inp):
+    gh, gw = w.grid
+    return O.forward(inp["q"], inp["k"], inp["v"], BIAS_KIND[w.bias], inp["bias"], inp["ld"], gh, gw)
+
+
+# ------------------------------------------------------------------ pre-passes
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_pack_and_quant_full_size(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    BH = w.B * w.H
+    for key in ("q", "k"):
+        x = _gpu(inp[key], w.dtype)
+        bits, mu = ba.pack_qk(x)
+        torch.cuda.synchronize()
+        ob, om = O.pack(inp[key].reshape(BH, w.N, w.d))
+        np.testing.assert_array_equal(_bits(bits).reshape(ob.shape), ob)
+        rel = np.abs(mu.cpu().numpy().reshape(om.shape).astype(np.float64) - om) / np.maximum(om, 1e-30)
+        assert rel.max() <= w.d * 2.0 ** -24 + 2.0 ** -23
+        del x, bits, mu
+    v = _gpu(inp["v"], w.dtype)
+    vq, sv = ba.quant_v(v)
+    torch.cuda.synchronize()
+    ovq, osv = O.quant_v(inp["v"].reshape(BH, w.N, w.d))
+    np.testing.assert_array_equal(sv.cpu().numpy().reshape(osv.shape), osv)
+    np.testing.assert_array_equal(_vq_natural(vq, w.N), ovq)
+    assert vq.shape[-1] == ba.vq_ld(w.N)
+    assert not vq[..., w.N:].any()
+
+
+@pytest.mark.parametrize("d", [1, 31, 33, 72, 96, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_pack_and_quant_odd_d(d, dtype):
+    w = Workload("odd", 2, 3, 77, d, dtype=dtype)
+    inp = make_inputs(w)
+    inp["q"][0, 0, 0, :] = 0.0
+    inp["q"][0, 0, 1, :] = -0.0
+    bits, mu = ba.pack_qk(_gpu(inp["q"], dtype))
+    vq, sv = ba.quant_v(_gpu(inp["v"], dtype))
+    torch.cuda.synchronize()
+    ob, om = O.pack(inp["q"].reshape(6, 77, d))
+    np.testing.assert_array_equal(_bits(bits).reshape(ob.shape), ob)
+    np.testing.assert_allclose(mu.cpu().numpy().reshape(om.shape), om, rtol=d * 2.0 ** -24 + 2.0 ** -23)
+    ovq, osv = O.quant_v(inp["v"].reshape(6, 77, d))
+    np.testing.assert_array_equal(_vq_natural(vq, 77), ovq)
+    np.testing.assert_array_equal(sv.cpu().numpy().reshape(osv.shape), osv)
+
+
+# ------------------------------------------------------------------ binary scores
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_scores_debug_bit_exact(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    bq, _ = ba.pack_qk(_gpu(inp["q"], w.dtype))
+    bk, _ = ba.pack_qk(_gpu(inp["k"], w.dtype))
+    ob, _ = O.pack(inp["q"].reshape(w.B * w.H, w.N, w.d))
+    okb, _ = O.pack(inp["k"].reshape(w.B * w.H, w.N, w.d))
+    Wd = ba.words(w.d)
+    heads = sorted({0, (w.B * w.H) // 2, w.B * w.H - 1})
+    rng = np.random.default_rng(1)
+    for bh in heads:
+        b, h = divmod(bh, w.H)
+        z = ba.scores_debug(bq[b:b + 1, h:h + 1].contiguous(), bk[b:b + 1, h:h + 1].contiguous(), w.d)
+        torch.cuda.synchronize()
+        rows = np.arange(w.N) if w.N <= 1024 else np.sort(rng.choice(w.N, 48, replace=False))
+        zo = O.scores_rows(ob[bh], okb[bh], w.d, rows)
+        np.testing.assert_array_equal(z[0, 0].cpu().numpy()[rows], zo)
+        del z
+    assert Wd == (w.d + 31) // 32
+
+
+# ------------------------------------------------------------------ attention
+
+SMALL = [
+    # name, B, H, N, d, dtype, bias, grid
+    ("tiles_ragged", 2, 3, 300, 64, "bf16", "dense", (0, 0)),
+    ("relpos", 1, 2, 300, 64, "bf16", "relpos2d", (15, 20)),
+    ("relpos_128", 1, 2, 384, 64, "bf16", "relpos2d", (3, 128)),
+    ("nobias_d72", 2, 2, 257, 72, "bf16", "none", (0, 0)),
+    ("f32_d64", 1, 3, 197, 64, "f32", "dense", (0, 0)),
+    ("n1", 2, 2, 1, 64, "bf16", "dense", (0, 0)),
+    ("n2", 1, 1, 2, 64, "f32", "none", (0, 0)),
+    ("n127", 1, 2, 127, 64, "bf16", "dense", (0, 0)),
+    ("n129", 1, 2, 129, 72, "bf16", "dense", (0, 0)),
+    ("d32", 1, 2, 200, 32, "bf16", "dense", (0, 0)),
+    ("d96", 1, 2, 150, 96, "f32", "dense", (0, 0)),
+    ("d128", 1, 1, 140, 128, "bf16", "none", (0, 0)),
+    ("d33", 1, 2, 90, 33, "f32", "dense", (0, 0)),
+    ("d1", 1, 1, 40, 1, "f32", "none", (0, 0)),
+]
+
+
+def _small_workload(spec):
+    name, B, H, N, d, dtype, bias, grid = spec
+    return Workload(name, B, H, N, d, dtype=dtype, bias=bias, grid=grid, bias_std=0.3)
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=[s[0] for s in SMALL])
+@pytest.mark.parametrize("variant", [NAT.BA_QK_AUTO, NAT.BA_QK_POPC] + TC_VARIANTS)
+def test_attention_small_cases(spec, variant):
+    w = _small_workload(spec)
+    inp = make_inputs(w)
+    try:
+        g = _run_gpu(w, inp, variant)
+    except NAT.BAError as e:
+        assert e.status == NAT.BA_ERR_UNSUPPORTED and variant in TC_VARIANTS
+        pytest.skip("variant does not take this shape")
+    ref = _oracle_full(w, inp)
+    _assert_close(g["out"].cpu().numpy(), ref["out"], inp["v"])
+    assert ba.check_device_status() == 0
+
+
+def test_attention_bf16_output_matches_f32_output():
+    w = _small_workload(SMALL[0])
+    inp = make_inputs(w)
+    a = _run_gpu(w, inp, out_dtype=torch.float32)["out"]
+    b = _run_gpu(w, inp, out_dtype=torch.bfloat16)["out"]
+    torch.testing.assert_close(b.float(), a.to(torch.bfloat16).float(), rtol=0, atol=0)
+
+
+def test_dominant_bias_selects_value_on_gpu():
+    """Special case on the GPU: a +100 bias entry per row picks one key."""
+    w = Workload("dom", 1, 2, 260, 64, bias="dense")
+    inp = make_inputs(w)
+    b = np.zeros_like(inp["bias"])
+    for i in range(w.N):
+        b[:, i, (5 * i + 1) % w.N] = 100.0
+    inp["bias"] = b
+    g = _run_gpu(w, inp)
+    ref = _oracle_full(w, inp)
+    _assert_close(g["out"].cpu().numpy(), ref["out"], inp["v"])
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_attention_full_size(name):
+    """Every workload at its full size, in the launch configuration the
+    benchmark times.  Small heads are compared in full; for the large ones the
+    oracle computes sampled rows one by one."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    g = _run_gpu(w, inp)
+    out = g["out"].cpu().numpy()
+    del g
+    torch.cuda.empty_cache()
+    gh, gw = w.grid
+    BH = w.B * w.H
+    kind = BIAS_KIND[w.bias]
+    if w.B * w.H * w.N * w.N <= 4e7:
+        ref = _oracle_full(w, inp)
+        _assert_close(out, ref["out"], inp["v"])
+        return
+    bq, muq = O.pack(inp["q"].reshape(BH, w.N, w.d))
+    bk, muk = O.pack(inp["k"].reshape(BH, w.N, w.d))
+    vq, sv = O.quant_v(inp["v"].reshape(BH, w.N, w.d))
+    rng = np.random.default_rng(2)
+    heads = sorted({0, BH // 3, BH - 1})
+    n_rows = w.N if w.N <= 1024 else 40
+    got, want, vs = [], [], []
+    for bh in heads:
+        rows = np.arange(w.N) if n_rows == w.N else np.sort(rng.choice(w.N, n_rows, replace=False))
+        for r in rows:
+            o, _, _, _ = O.attention_rows(bq, muq, bk, muk, vq, sv, kind, inp["bias"], inp["ld"], gh, gw,
+                                          w.H, bh, int(r), int(r) + 1, w.d)
+            want.append(o[0])
+            got.append(out.reshape(BH, w.N, w.d)[bh, r])
+        vs.append(np.broadcast_to(inp["v"].reshape(BH, w.N, w.d)[bh].std(axis=0), (len(rows), w.d)))
+    scale = np.maximum(1.0, np.concatenate(vs))
+    err = np.abs(np.array(got) - np.array(want)) / scale
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+
+
+def test_device_status_is_clean():
+    assert ba.check_device_status() == 0
