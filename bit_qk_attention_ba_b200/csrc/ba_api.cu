@@ -76,16 +76,18 @@ static bool sizes_ok(int B, int H, int N, int d)
            (int64_t)N <= (1 << 24);
 }
 
-static bool ptr_ok(const void* p) { return p != nullptr && aligned(p, 16); }
+// Non-null and aligned to `a` bytes.
+static bool ptr_ok(const void* p, uintptr_t a) { return p != nullptr && aligned(p, a); }
+static uintptr_t esize(ba_dtype dt) { return dt == BA_BF16 ? 2 : 4; }
 
 static ba_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BA_OK : BA_ERR_CUDA; }
 
 static bool bias_ok(int kind, const float* bias, int64_t ld, int gh, int gw, int N)
 {
     if (kind == BA_BIAS_NONE) return true;
-    if (kind == BA_BIAS_DENSE) return ptr_ok(bias) && ld >= N && ld % 4 == 0;
+    if (kind == BA_BIAS_DENSE) return ptr_ok(bias, 16) && ld >= N && ld % 4 == 0;
     if (kind == BA_BIAS_RELPOS2D)
-        return ptr_ok(bias) && gh >= 1 && gw >= 1 && (int64_t)gh * gw == N;
+        return ptr_ok(bias, 4) && gh >= 1 && gw >= 1 && (int64_t)gh * gw == N;
     return false;
 }
 
@@ -115,7 +117,7 @@ ba_status ba_pack_qk(const void* x, ba_dtype dt, int B, int H, int N, int d,
                      uint32_t* bits, float* mu, void* stream)
 {
     if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
-    if (!ptr_ok(x) || !ptr_ok(bits) || !ptr_ok(mu)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(x, esize(dt)) || !ptr_ok(bits, 4) || !ptr_ok(mu, 4)) return BA_ERR_INVALID_ARG;
     const int sms = sm_count();
     if (sms <= 0) return BA_ERR_CUDA;
     return from_cuda(launch_pack(x, dt, (int64_t)B * H * N, d, bits, mu,
@@ -126,7 +128,7 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
                      int8_t* vq, float* sv, void* stream)
 {
     if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
-    if (!ptr_ok(v) || !ptr_ok(vq) || !ptr_ok(sv)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(v, esize(dt)) || !ptr_ok(vq, 16) || !ptr_ok(sv, 4)) return BA_ERR_INVALID_ARG;
     return from_cuda(launch_quant_v(v, dt, B, H, N, d, vq, sv, static_cast<cudaStream_t>(stream)));
 }
 
@@ -134,7 +136,7 @@ ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, 
                           int32_t* z, void* stream)
 {
     if (!sizes_ok(B, H, N, d)) return BA_ERR_INVALID_ARG;
-    if (!ptr_ok(bq) || !ptr_ok(bk) || !ptr_ok(z)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq, 4) || !ptr_ok(bk, 4) || !ptr_ok(z, 4)) return BA_ERR_INVALID_ARG;
     if (ceil_div(N, 64) > 65535) return BA_ERR_UNSUPPORTED;
     return from_cuda(launch_scores(bq, bk, B, H, N, d, z, static_cast<cudaStream_t>(stream)));
 }
@@ -148,8 +150,8 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    void* out, ba_dtype out_dt, int variant, void* stream)
 {
     if (!sizes_ok(B, H, N, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
-    if (!ptr_ok(bq) || !ptr_ok(muq) || !ptr_ok(bk) || !ptr_ok(muk) || !ptr_ok(vq) || !ptr_ok(sv) ||
-        !ptr_ok(out))
+    if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
+        !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)))
         return BA_ERR_INVALID_ARG;
     if (!bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N)) return BA_ERR_INVALID_ARG;
     if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_TC_I8 && variant != BA_QK_TC_F8)

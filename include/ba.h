@@ -13,9 +13,11 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
- *     in the layout stated, and 16-byte aligned.  The library allocates no
- *     device memory and never synchronises: work is queued on `stream` (a
- *     cudaStream_t passed as void*; NULL is the legacy default stream).
+ *     in the layout stated and aligned to their element size; the int8 V codes
+ *     and a dense bias must be 16-byte aligned (they are read by the tensor
+ *     memory accelerator).  The library allocates no device memory and never
+ *     synchronises: work is queued on `stream` (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream).
  *   - Arguments are validated before anything is queued; an invalid call
  *     returns BA_ERR_INVALID_ARG (or BA_ERR_UNSUPPORTED) and queues nothing.
  *   - A launch failure reported by the CUDA runtime returns BA_ERR_CUDA.

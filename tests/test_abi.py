@@ -49,7 +49,7 @@ def test_pure_helpers(lib):
 
 
 FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced (validation fails first)
-MIS = ctypes.c_void_p((1 << 20) + 4)      # misaligned
+MIS = ctypes.c_void_p((1 << 20) + 1)      # misaligned for every element type
 
 
 @pytest.mark.parametrize("B,H,N,d", [(0, 1, 8, 64), (1, 0, 8, 64), (1, 1, 0, 64), (1, 1, 8, 0), (1, 1, 8, 129),

@@ -133,7 +133,7 @@ def test_scores_debug_bit_exact(name):
     rng = np.random.default_rng(1)
     for bh in heads:
         b, h = divmod(bh, w.H)
-        z = ba.scores_debug(bq[b:b + 1, h:h + 1].contiguous(), bk[b:b + 1, h:h + 1].contiguous(), w.d)
+        z = ba.scores_debug(bq[b:b + 1, h:h + 1], bk[b:b + 1, h:h + 1], w.d)   # views: 4-byte aligned
         torch.cuda.synchronize()
         rows = np.arange(w.N) if w.N <= 1024 else np.sort(rng.choice(w.N, 48, replace=False))
         zo = O.scores_rows(ob[bh], okb[bh], w.d, rows)
