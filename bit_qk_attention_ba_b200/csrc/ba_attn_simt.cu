@@ -1,11 +1,12 @@
 // ba_attn_simt.cu -- the BinaryAttention forward on CUDA cores only.
 //
 // QK variant "popc": every score is d - 2 popcount(XOR) over 32-bit words
-// (BA notes, Key design 1), scaled and biased (Key design 2), folded into a
-// FlashAttention2-style online softmax (Overall framework), P quantised to u8
-// with scale 1/255 and multiplied with the int8 V codes by dp4a (u8 x s8 ->
-// s32), Key design 3.  One thread owns one query row; a CTA walks the keys in
-// tiles of 32 staged in shared memory.  This is the plain, any-shape path and
+// (BA notes, Key design 1), scaled and biased (Key design 2).  The keys are
+// walked twice in tiles of 32 staged in shared memory (Overall framework):
+// the first sweep finds the exact row maximum, the second quantises
+// P~ = exp(S - m) to u8 with scale 1/255 and multiplies it with the int8 V
+// codes by dp4a (u8 x s8 -> s32), Key design 3.  One thread owns one query
+// row.  This is the plain, any-shape path and
 // the CUDA-core point of the QK variant comparison; the tensor-core kernel is
 // in ba_attn_tc.cu.
 #include <math.h>
@@ -62,68 +63,66 @@ attn_simt_kernel(const uint32_t* __restrict__ bq, const float* __restrict__ muq,
     for (int w = 0; w < W; ++w) q[w] = row_ok ? bq[(bh * N + i) * W + w] : 0u;
     const float cq = row_ok ? muq[bh * N + i] / sqrtf((float)d) : 0.f;
 
+    // Pass A: the exact row maximum.  Pass B: P~ = exp(S - m) against it, so
+    // the u8 codes need no later rescaling and the PV sum stays in int32.
     float m = -INFINITY, l = 0.f;
-    float o[DV];
+    int acc[DV];
 #pragma unroll
-    for (int c = 0; c < DV; ++c) o[c] = 0.f;
+    for (int c = 0; c < DV; ++c) acc[c] = 0;
 
-    for (int j0 = 0; j0 < N; j0 += KT) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < KT * W; idx += blockDim.x) {
-            const int r = idx / W, w = idx - r * W;
-            s_k[r][w] = (j0 + r < N) ? bk[(bh * N + j0 + r) * W + w] : 0u;
-        }
-        if (threadIdx.x < KT) s_muk[threadIdx.x] = (j0 + threadIdx.x < N) ? muk[bh * N + j0 + threadIdx.x] : 0.f;
-        for (int idx = threadIdx.x; idx < DV * 2; idx += blockDim.x) {   // two 16-byte halves per channel
-            const int c = idx >> 1, half = idx & 1;
-            const int64_t col = (int64_t)j0 + half * 16;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (c < d && col < ldv) val = *reinterpret_cast<const uint4*>(vq + (bh * d + c) * ldv + col);
-            *reinterpret_cast<uint4*>(&s_v[c][half * 4]) = val;
-        }
-        __syncthreads();
-
-        float s[KT];
-        float mt = -INFINITY;
-#pragma unroll
-        for (int jj = 0; jj < KT; ++jj) {
-            const int j = j0 + jj;
-            float val = -INFINITY;
-            if (j < N) {
-                int ham = 0;
-#pragma unroll
-                for (int w = 0; w < W; ++w) ham += __popc(q[w] ^ s_k[jj][w]);
-                const float z = (float)(d - 2 * ham);
-                const float b = row_ok ? bias_at(bias_kind, bias, bias_ld, h, N, gh, gw, i, j) : 0.f;
-                val = fmaf(cq * s_muk[jj], z, b);
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int j0 = 0; j0 < N; j0 += KT) {
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < KT * W; idx += blockDim.x) {
+                const int r = idx / W, w = idx - r * W;
+                s_k[r][w] = (j0 + r < N) ? bk[(bh * N + j0 + r) * W + w] : 0u;
             }
-            s[jj] = val;
-            mt = fmaxf(mt, val);
-        }
-        const float m_new = fmaxf(m, mt);
-        const float alpha = expf(m - m_new);     // 0 on the first tile (m = -inf)
-        l *= alpha;
-#pragma unroll
-        for (int c = 0; c < DV; ++c) o[c] *= alpha;
+            if (threadIdx.x < KT) s_muk[threadIdx.x] = (j0 + threadIdx.x < N) ? muk[bh * N + j0 + threadIdx.x] : 0.f;
+            if (pass == 1) {
+                for (int idx = threadIdx.x; idx < DV * 2; idx += blockDim.x) {   // two 16-byte halves per channel
+                    const int c = idx >> 1, half = idx & 1;
+                    const int64_t col = (int64_t)j0 + half * 16;
+                    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+                    if (c < d && col < ldv) val = *reinterpret_cast<const uint4*>(vq + (bh * d + c) * ldv + col);
+                    *reinterpret_cast<uint4*>(&s_v[c][half * 4]) = val;
+                }
+            }
+            __syncthreads();
 
-        uint32_t pw[KT / 4];
+            float s[KT];
 #pragma unroll
-        for (int w = 0; w < KT / 4; ++w) pw[w] = 0u;
+            for (int jj = 0; jj < KT; ++jj) {
+                const int j = j0 + jj;
+                float val = -INFINITY;
+                if (j < N) {
+                    int ham = 0;
 #pragma unroll
-        for (int jj = 0; jj < KT; ++jj) {
-            const float p = expf(s[jj] - m_new);
-            l += p;
-            const uint32_t pq = (uint32_t)__float2int_rn(255.f * p);
-            pw[jj >> 2] |= pq << (8 * (jj & 3));
+                    for (int w = 0; w < W; ++w) ham += __popc(q[w] ^ s_k[jj][w]);
+                    const float z = (float)(d - 2 * ham);
+                    const float b = row_ok ? bias_at(bias_kind, bias, bias_ld, h, N, gh, gw, i, j) : 0.f;
+                    val = fmaf(cq * s_muk[jj], z, b);
+                }
+                s[jj] = val;
+                if (pass == 0) m = fmaxf(m, val);
+            }
+            if (pass == 0) continue;
+
+            uint32_t pw[KT / 4];
+#pragma unroll
+            for (int w = 0; w < KT / 4; ++w) pw[w] = 0u;
+#pragma unroll
+            for (int jj = 0; jj < KT; ++jj) {
+                const float p = expf(s[jj] - m);
+                l += p;
+                const uint32_t pq = (uint32_t)__float2int_rn(255.f * p);
+                pw[jj >> 2] |= pq << (8 * (jj & 3));
+            }
+#pragma unroll
+            for (int c = 0; c < DV; ++c) {
+#pragma unroll
+                for (int w = 0; w < KT / 4; ++w) acc[c] = dp4a_u8s8(pw[w], s_v[c][w], acc[c]);
+            }
         }
-#pragma unroll
-        for (int c = 0; c < DV; ++c) {
-            int acc = 0;
-#pragma unroll
-            for (int w = 0; w < KT / 4; ++w) acc = dp4a_u8s8(pw[w], s_v[c][w], acc);
-            o[c] += (float)acc;
-        }
-        m = m_new;
     }
 
     if (row_ok) {
@@ -131,7 +130,7 @@ attn_simt_kernel(const uint32_t* __restrict__ bq, const float* __restrict__ muq,
         OutT* dst = out + (bh * N + i) * d;
 #pragma unroll
         for (int c = 0; c < DV; ++c)
-            if (c < d) store_out<OutT>(dst + c, sv[bh * d + c] * o[c] * inv);
+            if (c < d) store_out<OutT>(dst + c, sv[bh * d + c] * (float)acc[c] * inv);
     }
 }
 

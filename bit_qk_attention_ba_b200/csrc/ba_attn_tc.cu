@@ -4,32 +4,44 @@
 // Vision and Diffusion Transformers", CVPR 2026):
 //   Key design 1: s_i . t_j from sign bits, per-token scales mu
 //   Key design 2: S_ij = mu_q,i mu_k,j s_i.t_j / sqrt(d) + b_ij
-//   Key design 3: P~ as u8 with scale 1/255, int8 V per channel, integer PV
-//   Overall framework: FlashAttention2-style tiling with an online softmax.
+//   Key design 3: P~ = exp(S - m) as u8 with scale 1/255, channel-wise int8
+//                 V, integer PV product
+//   Overall framework: a tiled attention in the FlashAttention2 style.
 //
-// The A100 design on the page (mma.sync .b1 for QK, mma.sync u8.s8 for PV) is
-// prior art; this kernel is built for Blackwell instead:
-//   * one CTA per 128-query tile (M = 128 = TMEM lanes, one softmax thread per
-//     query row, so row max / row sum need no shuffles);
-//   * QK on tcgen05.mma with the sign bits expanded to +-1 operands in shared
-//     memory (kind::i8 -> s32, or kind::f8f6f4 with e4m3 +-1 -> f32; both
-//     exact), accumulating S in TMEM, double-buffered so QK of the next key
-//     tile overlaps the softmax of this one;
-//   * PV on tcgen05.mma kind::i8 with u8 P and s8 V (K-major int8 V tiles
-//     brought in by TMA with 128-byte swizzle), the s32 accumulator living in
-//     TMEM across all key tiles;
-//   * the online softmax keeps m and l in registers; when a warp's running
-//     maxima move, that warp rescales its accumulator rows in TMEM with a
-//     fixed-point multiply (exact to half a unit);
-//   * a dense bias tile is staged by TMA (128-byte swizzle, conflict-free
-//     reads); a 2-D relative-position bias is gathered from the per-head table
-//     through a per-key offset the load warp precomputes.
-// Warp roles: warp 0 loads (TMA + sign-bit expansion), warp 1 issues MMAs and
-// owns TMEM, warps 2..5 run the softmax and the epilogue.
+// The A100 design on the page (mma.sync .b1 for QK, mma.sync u8.s8 for PV,
+// one pass with a running maximum) is prior art.  This kernel is built for
+// Blackwell:
+//   * a CTA owns two groups of 128 query rows, one softmax thread per query
+//     row (row = TMEM lane), so row reductions need no shuffles.  With a
+//     dense bias the groups are the same rows of two batch elements, so one
+//     bias tile serves both; otherwise they are two row blocks of one head,
+//     so one key/value tile serves both;
+//   * the keys are swept twice: pass A finds the exact row maximum m_i, pass
+//     B quantises P~ = exp(S - m_i) against it.  The u8 codes are then the
+//     ones an exact-maximum reference produces, and the int32 PV accumulator
+//     never needs rescaling;
+//   * QK runs on tcgen05.mma from sign bits expanded to +-1 operands in shared
+//     memory (kind::i8 -> s32, or kind::f8f6f4 with e4m3 +-1 -> f32; both are
+//     exact), into double-buffered S tiles in TMEM, so the next tile's QK
+//     overlaps this tile's softmax;
+//   * PV runs on tcgen05.mma kind::i8 (u8 P from shared memory, s8 V tiles
+//     brought in by TMA), accumulating in TMEM across all key tiles;
+//   * the softmax pulls each 64-key S tile out of TMEM with one load and does
+//     its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with a 3-input
+//     max;
+//   * the loaders fetch a step's sign bits, scales and bias values into
+//     registers two steps ahead, so global latency overlaps the wait for a
+//     free stage; 2 to 4 stages, as shared memory allows;
+//   * a dense bias tile is staged by TMA with 128-byte swizzle; a 2-D
+//     relative-position bias whose grid width is a multiple of 128 is staged
+//     as reversed, shifted copies of the one table row the tile needs, so each
+//     thread reads its bias as aligned 16-byte vectors.
+// Warps 0-7 run the softmax (two groups of four), warps 8-11 load, warp 12
+// issues the MMAs and owns TMEM.
 //
 // Every wait on an mbarrier is bounded; on a timeout the kernel records a bit
-// in the device status word, tells the other roles to stop, lets in-flight
-// tensor-core work drain, frees TMEM and returns.
+// in the device status word, tells the other roles to stop, lets issued TMA
+// and tensor-core work drain, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -42,47 +54,71 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;          // query rows per CTA (= TMEM lanes)
-constexpr int BN = 128;          // keys per tile
-constexpr int STAGES = 2;        // key/value/bias buffers
-constexpr int NUM_THREADS = 192;
+constexpr int BM = 128;                 // query rows per group (= TMEM lanes)
+constexpr int NG = 2;                   // row groups per CTA
+constexpr int BN = 64;                  // keys per tile
+constexpr int MAX_STAGES = 4;
+constexpr int NUM_SOFTMAX_WARPS = 4 * NG;
+constexpr int NUM_LOAD_WARPS = 4;
+constexpr int NUM_LOADERS = 32 * NUM_LOAD_WARPS;
+constexpr int LOAD_WARP0 = NUM_SOFTMAX_WARPS;               // 8
+constexpr int MMA_WARP = LOAD_WARP0 + NUM_LOAD_WARPS;       // 12
+constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 416
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int QK_I8 = 0, QK_F8 = 1;
+constexpr int RP_SPAN = BM + BN - 2;    // largest offset inside a rel-pos window (190)
+constexpr int RP_VALS = RP_SPAN + 1;    // values in a window
+constexpr int RP_WIN = 192;             // entries per shifted copy of a window (RP_STRIDE >= RP_WIN)
+constexpr int RP_STRIDE = 200;          // floats between copies (8 words mod 32: conflict-free)
+constexpr int RP_PER_THREAD = (NG * RP_VALS + NUM_LOADERS - 1) / NUM_LOADERS;   // 3
 
 // Barrier slots.
 enum {
-    B_Q = 0,
-    B_SFULL = 1,     // 2: S tile in TMEM buffer b ready
-    B_SEMPTY = 3,    // 2: softmax has read S buffer b
-    B_PFULL = 5,     // P tile written (and accumulator rescaled)
-    B_PVDONE = 6,    // PV of the tile finished
-    B_KFULL = 7,     // STAGES: K operand, mu_k, key offsets ready
-    B_VFULL = 9,     // STAGES: V (and dense bias) TMA landed
-    B_KVEMPTY = 11,  // STAGES: stage may be overwritten
-    B_FINAL = 13,
-    NUM_BARS = 14
+    B_QREADY = 0,
+    B_FULL = 1,                      // [stage] operands, scales, bias (and V in pass B) ready
+    B_EMPTY = B_FULL + MAX_STAGES,   // [stage] stage may be overwritten
+    B_SFULL = B_EMPTY + MAX_STAGES,  // [NG][2] S tile in TMEM ready
+    B_SEMPTY = B_SFULL + 2 * NG,     // [NG][2] softmax done with S buffer
+    B_PFULL = B_SEMPTY + 2 * NG,     // [NG][2] u8 P tile written
+    B_PFREE = B_PFULL + 2 * NG,      // [NG][2] PV that read P buffer finished
+    B_FINAL = B_PFREE + 2 * NG,
+    NUM_BARS
 };
 
 struct Layout {
-    uint32_t v[STAGES], b[STAGES], q, k[STAGES], p, muk[STAGES], koff[STAGES], bars, misc, total;
+    uint32_t stages, kvg;       // pipeline depth; key/value sets per stage (1 or 2)
+    uint32_t v, v_bytes;        // [stage][kvg] V tiles (SW64 K-major, dv rows x 64 bytes)
+    uint32_t b;                 // [stage][2] dense bias boxes, 16 KB each (SW128)
+    uint32_t q, q_bytes;        // [NG] Q operands
+    uint32_t k, k_bytes;        // [stage][kvg] K operands
+    uint32_t p;                 // [NG][2] P tiles, 8 KB each
+    uint32_t muk, koff;         // [stage][kvg][BN], [stage][BN]
+    uint32_t rp;                // [stage][NG][4][RP_STRIDE] rel-pos windows
+    uint32_t bars, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Layout make_layout(int dpad, int dv, bool dense_bias)
+__host__ __device__ inline Layout make_layout(int dpad, int dv, int bias_kind, int stages)
 {
     Layout L;
+    L.stages = stages;
+    L.kvg = (bias_kind == BA_BIAS_DENSE) ? 2u : 1u;
     uint32_t off = 0;
-    for (int s = 0; s < STAGES; ++s) { (s ? L.v[1] : L.v[0]) = off; off = align_up(off + dv * 128u, 1024); }
-    for (int s = 0; s < STAGES; ++s) { (s ? L.b[1] : L.b[0]) = off; off = align_up(off + (dense_bias ? 4u * 16384u : 0u), 1024); }
-    L.q = off; off = align_up(off + BM * (uint32_t)dpad, 1024);
-    for (int s = 0; s < STAGES; ++s) { (s ? L.k[1] : L.k[0]) = off; off = align_up(off + BN * (uint32_t)dpad, 1024); }
-    L.p = off; off = align_up(off + BM * BN, 1024);
-    for (int s = 0; s < STAGES; ++s) { (s ? L.muk[1] : L.muk[0]) = off; off += BN * 4; }
-    for (int s = 0; s < STAGES; ++s) { (s ? L.koff[1] : L.koff[0]) = off; off += BN * 4; }
+    L.v_bytes = align_up((uint32_t)dv * BN, 1024);
+    L.v = off; off += stages * L.kvg * L.v_bytes;
+    L.b = off; off += (bias_kind == BA_BIAS_DENSE) ? stages * 2 * 16384u : 0u;
+    L.q_bytes = align_up((uint32_t)BM * dpad, 1024);
+    L.q = off; off += NG * L.q_bytes;
+    L.k_bytes = align_up((uint32_t)BN * dpad, 1024);
+    L.k = off; off += stages * L.kvg * L.k_bytes;
+    L.p = off; off += NG * 2 * BM * BN;
+    L.muk = off; off += stages * L.kvg * BN * 4;
+    L.koff = off; off += stages * BN * 4;
+    L.rp = off; off += (bias_kind == BA_BIAS_RELPOS2D) ? stages * NG * 4 * RP_STRIDE * 4u : 0u;
     L.bars = off; off += NUM_BARS * 8;
-    L.misc = off; off += 16;        // TMEM base address, abort flag
+    L.misc = off; off += 16;            // TMEM base address, abort flag
     L.total = off;
     return L;
 }
@@ -95,14 +131,14 @@ struct Params {
     const float* sv;
     const float* table;      // 2-D relative-position table (global)
     void* out;
-    int H, N, d, W, dpad, dv, n_tiles;
-    int gh, gw;
+    int B, H, N, d, W, dpad, dv, n_tiles, stages;
+    int gh, gw, relpos_fast;
     float q_scale;           // 1 / sqrt(d)
     unsigned* status;
 };
 
-// 16 sign bits -> 16 bytes of +-1 operands (+1 where the bit is set), with
-// byte lanes whose bit in `valid` is 0 forced to 0 (padding channels).
+// 16 sign bits -> 16 bytes of +-1 operands (+1 where the bit is set); byte
+// lanes whose bit in `valid` is 0 are forced to 0 (padding channels).
 template <int QK>
 __device__ __forceinline__ uint4 expand16(uint32_t bits, uint32_t valid)
 {
@@ -127,15 +163,15 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// Byte offset of (row r, 16-byte chunk kc) in a K-major, non-swizzled
-// operand whose rows hold `chunks` 16-byte chunks: 8x16-byte core matrices,
-// chunk-adjacent core matrices 128 bytes apart, 8-row groups chunks*128 apart.
+// Byte offset of (row r, 16-byte chunk kc) in a K-major, non-swizzled operand
+// whose rows hold `chunks` 16-byte chunks: 8 x 16-byte core matrices, chunk
+// neighbours 128 bytes apart, 8-row groups chunks * 128 bytes apart.
 __device__ __forceinline__ uint32_t core_off(int r, int kc, int chunks)
 {
     return (uint32_t)((r >> 3) * chunks * 128 + kc * 128 + (r & 7) * 16);
 }
 
-// Warp-uniform bounded wait: every lane polls; all agree on the outcome.
+// Warp-uniform bounded wait: every lane polls, all agree on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
 {
     const bool ok = mbar_wait(bar, parity, abort_flag);
@@ -152,48 +188,154 @@ template <typename OutT> __device__ __forceinline__ void store1(OutT* p, float v
 template <> __device__ __forceinline__ void store1<float>(float* p, float v) { *p = v; }
 template <> __device__ __forceinline__ void store1<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// Which (batch*head, first query row) a row group of this CTA covers, and
+// whether that group exists.  Dense bias: groups are batch elements 2z and
+// 2z+1 of head y, rows 128x.  Otherwise: rows 256x and 256x+128 of head y.
+template <bool PAIR>
+__device__ __forceinline__ void group_coords(const Params& p, int g, int& bh, int& q0, bool& exists)
+{
+    if (PAIR) {
+        int b = 2 * blockIdx.z + g;
+        exists = b < p.B;
+        if (!exists) b = p.B - 1;
+        bh = b * p.H + blockIdx.y;
+        q0 = blockIdx.x * BM;
+    } else {
+        bh = blockIdx.y;
+        q0 = blockIdx.x * (BM * NG) + g * BM;
+        exists = q0 < p.N;
+    }
+}
+
+// One 64-key tile of one row: S = z * mu_k * cq + b (Key design 2) on packed
+// pairs, then either the row maximum (pass A) or P~ = exp(S - m), the row sum
+// and the u8 codes round(255 P~) (pass B).  MASK drops keys >= N.  Two
+// independent max / sum accumulators keep the dependency chains short.
+template <int QK, int BIAS, bool PASS_B, bool MASK>
+__device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const float* mks, const uint8_t* bsm_row,
+                                             int bsm_sw, const float* rp_copy, const int* koff,
+                                             const float* tab_h, int rel_base, int nvalid,
+                                             uint64_t cq2, uint64_t neg2, float (&mx)[2], uint64_t (&l2)[2],
+                                             uint32_t (&pw)[16])
+{
+    const uint64_t L2E = f2_pack(LOG2E, LOG2E);
+    const uint64_t C255 = f2_pack(255.f, 255.f);
+    const uint64_t MAGIC = f2_pack(12582912.f, 12582912.f);
+#pragma unroll
+    for (int k4 = 0; k4 < BN / 4; ++k4) {
+        const float4 mk = *reinterpret_cast<const float4*>(mks + 4 * k4);
+        float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (BIAS == BA_BIAS_DENSE) {
+            bb = *reinterpret_cast<const float4*>(bsm_row + (k4 >> 3) * 16384 + (((k4 & 7) ^ bsm_sw) << 4));
+        } else if (BIAS == BA_BIAS_RELPOS2D) {
+            if (rp_copy) {
+                bb = *reinterpret_cast<const float4*>(rp_copy + 4 * k4);
+            } else {
+                const int4 ko = *reinterpret_cast<const int4*>(koff + 4 * k4);
+                bb = make_float4(__ldg(tab_h + rel_base - ko.x), __ldg(tab_h + rel_base - ko.y),
+                                 __ldg(tab_h + rel_base - ko.z), __ldg(tab_h + rel_base - ko.w));
+            }
+        }
+        uint64_t z01, z23;
+        if (QK == QK_F8) {
+            z01 = f2_pack(__uint_as_float(zr[4 * k4]), __uint_as_float(zr[4 * k4 + 1]));
+            z23 = f2_pack(__uint_as_float(zr[4 * k4 + 2]), __uint_as_float(zr[4 * k4 + 3]));
+        } else {   // s32 -> f32 exactly: |z| < 2^22, so 1.5 * 2^23 + z is exact
+            const uint64_t NM = f2_pack(-12582912.f, -12582912.f);
+            z01 = f2_add(f2_pack(__uint_as_float(zr[4 * k4] + 0x4B400000u),
+                                 __uint_as_float(zr[4 * k4 + 1] + 0x4B400000u)), NM);
+            z23 = f2_add(f2_pack(__uint_as_float(zr[4 * k4 + 2] + 0x4B400000u),
+                                 __uint_as_float(zr[4 * k4 + 3] + 0x4B400000u)), NM);
+        }
+        uint64_t s01 = f2_fma(f2_mul(z01, f2_pack(mk.x, mk.y)), cq2, f2_pack(bb.x, bb.y));
+        uint64_t s23 = f2_fma(f2_mul(z23, f2_pack(mk.z, mk.w)), cq2, f2_pack(bb.z, bb.w));
+        if (MASK) {
+            float a, b, c, e;
+            f2_unpack(s01, a, b);
+            f2_unpack(s23, c, e);
+            const int j = 4 * k4;
+            a = (j < nvalid) ? a : -INFINITY;
+            b = (j + 1 < nvalid) ? b : -INFINITY;
+            c = (j + 2 < nvalid) ? c : -INFINITY;
+            e = (j + 3 < nvalid) ? e : -INFINITY;
+            s01 = f2_pack(a, b);
+            s23 = f2_pack(c, e);
+        }
+        if (!PASS_B) {
+            float a, b, c, e;
+            f2_unpack(s01, a, b);
+            f2_unpack(s23, c, e);
+            mx[k4 & 1] = fmax3(mx[k4 & 1], a, b);
+            mx[k4 & 1] = fmax3(mx[k4 & 1], c, e);
+        } else {
+            float a, b, c, e;
+            f2_unpack(f2_fma(s01, L2E, neg2), a, b);
+            f2_unpack(f2_fma(s23, L2E, neg2), c, e);
+            const uint64_t p01 = f2_pack(ex2(a), ex2(b));
+            const uint64_t p23 = f2_pack(ex2(c), ex2(e));
+            l2[k4 & 1] = f2_add(l2[k4 & 1], f2_add(p01, p23));
+            float q0, q1, q2, q3;                      // low byte = round-half-even(255 P~)
+            f2_unpack(f2_fma(p01, C255, MAGIC), q0, q1);
+            f2_unpack(f2_fma(p23, C255, MAGIC), q2, q3);
+            pw[k4] = __byte_perm(__byte_perm(__float_as_uint(q0), __float_as_uint(q1), 0x0040),
+                                 __byte_perm(__float_as_uint(q2), __float_as_uint(q3), 0x0040), 0x5410);
+        }
+    }
+}
+
+// What one loader thread fetches from global memory for one step, held in
+// registers until the stage is free.
+struct Prefetch {
+    uint32_t kbits[4];           // sign words for up to 4 (key, word) items
+    float muk;                   // one key scale
+    int koff;                    // one key's rel-pos offset (general rel-pos path)
+    float rp[RP_PER_THREAD];     // rel-pos window values
+};
+
 template <int QK, typename OutT, int BIAS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
                const Params p)
 {
+    constexpr bool PAIR = (BIAS == BA_BIAS_DENSE);
+    constexpr int KVG = PAIR ? 2 : 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const Layout L = make_layout(p.dpad, p.dv, BIAS == BA_BIAS_DENSE);
+    const Layout L = make_layout(p.dpad, p.dv, BIAS, p.stages);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
-    const int h = bh % p.H;
-    const int q0 = blockIdx.x * BM;
-    const int N = p.N, W = p.W, T = p.n_tiles;
+    const int N = p.N, W = p.W, T = p.n_tiles, U = 2 * T;   // steps: pass A then pass B
+    const int S = p.stages;
     const int chunks = p.dpad / 16;
+    const int h = PAIR ? (int)blockIdx.y : (int)(blockIdx.y % p.H);
+    const float* tab_h = (BIAS == BA_BIAS_RELPOS2D)
+                             ? p.table + (size_t)h * (2 * p.gh - 1) * (2 * p.gw - 1) : nullptr;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[B_Q], 4);
-        for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars[B_QREADY], NUM_SOFTMAX_WARPS);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bars[B_FULL + s], NUM_LOAD_WARPS);
+            mbar_init(&bars[B_EMPTY + s], NUM_SOFTMAX_WARPS + 1);
+        }
+        for (int b = 0; b < 2 * NG; ++b) {
             mbar_init(&bars[B_SFULL + b], 1);
             mbar_init(&bars[B_SEMPTY + b], 4);
-        }
-        mbar_init(&bars[B_PFULL], 4);
-        mbar_init(&bars[B_PVDONE], 1);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&bars[B_KFULL + s], 1);
-            mbar_init(&bars[B_VFULL + s], 1);
-            mbar_init(&bars[B_KVEMPTY + s], 1);
+            mbar_init(&bars[B_PFULL + b], 4);
+            mbar_init(&bars[B_PFREE + b], 1);
         }
         mbar_init(&bars[B_FINAL], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == LOAD_WARP0 && lane == 0) {
         prefetch_tmap(&tm_v);
         if (BIAS == BA_BIAS_DENSE) prefetch_tmap(&tm_b);
     }
@@ -202,117 +344,224 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ loads
-        for (int t = 0; t < T; ++t) {
-            const int s = t % STAGES, use = t / STAGES;
-            if (t >= STAGES && !warp_wait(&bars[B_KVEMPTY + s], (use - 1) & 1, abort_flag)) {
-                if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutProducer);
-                break;
+    if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
+        // ---------------------------------------------------------------- loaders
+        // Every loader thread owns fixed items of each stage: up to four (key
+        // set, key, word) sign words, one key scale, and up to three values of
+        // the rel-pos windows.  Their addresses are worked out once here; per
+        // step only the key offset j0 moves.  Global loads for step u + 2 are
+        // issued right after step u is stored, so their latency overlaps the
+        // wait for a free stage.
+        const int lw = warp - LOAD_WARP0;
+        const int ltid = lw * 32 + lane;
+        int kvbh0, kvbh1;
+        {
+            int q0x;
+            bool ex;
+            group_coords<PAIR>(p, 0, kvbh0, q0x, ex);
+            kvbh1 = kvbh0;
+            if (KVG > 1) group_coords<PAIR>(p, 1, kvbh1, q0x, ex);
+        }
+        const int kitems = KVG * BN * W;
+        const uint32_t* kbase[4];
+        int krow[4];
+        uint32_t kdst[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int e = ltid + k * NUM_LOADERS;
+            const int x = e / (BN * W), rem = e - x * (BN * W);
+            const int r = rem / W, w = rem - r * W;
+            krow[k] = (e < kitems) ? r : (1 << 30);          // never valid
+            kbase[k] = p.bk + ((size_t)(x ? kvbh1 : kvbh0) * N + r) * W + w;
+            kdst[k] = (uint32_t)(x * L.k_bytes) + core_off(r, 2 * w, chunks);
+        }
+        const bool has_mu = ltid < KVG * BN;
+        const int mu_row = ltid % BN;
+        const float* mu_base = p.muk + (size_t)((ltid / BN) ? kvbh1 : kvbh0) * N + mu_row;
+        const float* rp_src[RP_PER_THREAD];
+        int rp_dst[RP_PER_THREAD], rp_v[RP_PER_THREAD];
+#pragma unroll
+        for (int k = 0; k < RP_PER_THREAD; ++k) {
+            const int e = ltid + k * NUM_LOADERS;
+            rp_v[k] = -1;
+            rp_src[k] = tab_h;
+            rp_dst[k] = 0;
+            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast && e < NG * RP_VALS) {
+                const int g = e / RP_VALS, v = e - g * RP_VALS;
+                int bhg, q0g;
+                bool ex;
+                group_coords<PAIR>(p, g, bhg, q0g, ex);
+                if (q0g >= N) q0g = N - BM;              // an empty group still reads inside the table
+                const int ri = q0g / p.gw, ci0 = q0g - ri * p.gw;
+                // Rr[v] = R[xlo + RP_SPAN - v] with R the table row of offset
+                // ri - rj and xlo = ci0 - cj0 - (BN - 1) + gw - 1; only the
+                // key-tile part rj * (2 gw - 1) + cj0 changes per step.
+                rp_src[k] = tab_h + (ptrdiff_t)(ri + p.gh - 1) * (2 * p.gw - 1) + ci0 - (BN - 1) + p.gw - 1 + RP_SPAN - v;
+                rp_v[k] = v;
+                rp_dst[k] = g * 4 * RP_STRIDE + v;
             }
+        }
+
+        auto fetch = [&](int u, Prefetch& f) {
+            const int t = (u >= T) ? u - T : u;
             const int j0 = t * BN;
-            if (lane == 0) {
-                const uint32_t bytes = (uint32_t)p.dv * 128u + (BIAS == BA_BIAS_DENSE ? 4u * 16384u : 0u);
-                mbar_arrive_expect_tx(&bars[B_VFULL + s], bytes);
-                tma_load_3d(smem + (s ? L.v[1] : L.v[0]), &tm_v, &bars[B_VFULL + s], j0, 0, bh);
-                if (BIAS == BA_BIAS_DENSE)
-                    for (int b = 0; b < 4; ++b)
-                        tma_load_3d(smem + (s ? L.b[1] : L.b[0]) + b * 16384, &tm_b, &bars[B_VFULL + s], j0 + 32 * b, q0, h);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                f.kbits[k] = (j0 + krow[k] < N) ? __ldg(kbase[k] + (size_t)j0 * W) : 0u;
+            f.muk = (has_mu && j0 + mu_row < N) ? __ldg(mu_base + j0) : 0.f;
+            f.koff = 0;
+            if (BIAS == BA_BIAS_RELPOS2D && !p.relpos_fast && ltid < BN) {
+                const int jj = min(j0 + ltid, N - 1);
+                const int rj = jj / p.gw, cj = jj - rj * p.gw;
+                f.koff = rj * (2 * p.gw - 1) + cj;
             }
-            uint8_t* kop = smem + (s ? L.k[1] : L.k[0]);
-            float* muk_s = reinterpret_cast<float*>(smem + (s ? L.muk[1] : L.muk[0]));
-            int* koff_s = reinterpret_cast<int*>(smem + (s ? L.koff[1] : L.koff[0]));
-            for (int r = lane; r < BN; r += 32) {
-                const int j = j0 + r;
-                const bool valid = j < N;
-                const uint32_t* src = p.bk + ((size_t)bh * N + j) * W;
-                for (int w = 0; w < W; ++w) {
-                    const uint32_t bits = valid ? __ldg(src + w) : 0u;
-                    *reinterpret_cast<uint4*>(kop + core_off(r, 2 * w, chunks)) = expand16<QK>(bits & 0xFFFFu, 0xFFFFu);
-                    *reinterpret_cast<uint4*>(kop + core_off(r, 2 * w + 1, chunks)) = expand16<QK>(bits >> 16, 0xFFFFu);
+            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast) {
+                const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
+                const ptrdiff_t shift = (ptrdiff_t)rj * (2 * p.gw - 1) + cj0;
+#pragma unroll
+                for (int k = 0; k < RP_PER_THREAD; ++k)
+                    f.rp[k] = (rp_v[k] >= 0) ? __ldg(rp_src[k] - shift) : 0.f;
+            }
+        };
+
+        auto step = [&](int u, const Prefetch& f) -> bool {
+            const int s = u % S, use = u / S;
+            const bool pass_b = u >= T;
+            const int t = pass_b ? u - T : u;
+            const int j0 = t * BN;
+            if (u >= S && !warp_wait(&bars[B_EMPTY + s], (use - 1) & 1, abort_flag)) {
+                if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutProducer);
+                return false;
+            }
+            if (lw == 0 && lane == 0) {
+                const uint32_t bytes = (pass_b ? (uint32_t)(KVG * p.dv * BN) : 0u) +
+                                       (BIAS == BA_BIAS_DENSE ? 2 * 16384u : 0u);
+                if (bytes) mbar_expect_tx(&bars[B_FULL + s], bytes);
+                if (pass_b) {
+                    tma_load_3d(smem + L.v + (s * KVG) * L.v_bytes, &tm_v, &bars[B_FULL + s], j0, 0, kvbh0);
+                    if (KVG > 1)
+                        tma_load_3d(smem + L.v + (s * KVG + 1) * L.v_bytes, &tm_v, &bars[B_FULL + s], j0, 0, kvbh1);
                 }
-                muk_s[r] = valid ? __ldg(p.muk + (size_t)bh * N + j) : 0.f;
-                if (BIAS == BA_BIAS_RELPOS2D) {
-                    const int jj = valid ? j : N - 1;
-                    const int rj = jj / p.gw, cj = jj - rj * p.gw;
-                    koff_s[r] = rj * (2 * p.gw - 1) + cj;
+                if (BIAS == BA_BIAS_DENSE)
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_3d(smem + L.b + (s * 2 + bx) * 16384, &tm_b, &bars[B_FULL + s],
+                                    j0 + 32 * bx, (int)blockIdx.x * BM, h);
+            }
+            uint8_t* kop = smem + L.k + s * KVG * L.k_bytes;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (krow[k] < BN) {
+                    *reinterpret_cast<uint4*>(kop + kdst[k]) = expand16<QK>(f.kbits[k] & 0xFFFFu, 0xFFFFu);
+                    *reinterpret_cast<uint4*>(kop + kdst[k] + 128) = expand16<QK>(f.kbits[k] >> 16, 0xFFFFu);
+                }
+            }
+            if (has_mu) {
+                reinterpret_cast<float*>(smem + L.muk)[s * KVG * BN + ltid] = f.muk;
+                if (BIAS == BA_BIAS_RELPOS2D && !p.relpos_fast && ltid < BN)
+                    reinterpret_cast<int*>(smem + L.koff)[s * BN + ltid] = f.koff;
+            }
+            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast) {
+                // Copy m of group g holds Rr[y + m]: value Rr[v] goes to y = v - m.
+                float* rp = reinterpret_cast<float*>(smem + L.rp) + (size_t)s * NG * 4 * RP_STRIDE;
+#pragma unroll
+                for (int k = 0; k < RP_PER_THREAD; ++k) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        if (rp_v[k] >= m) rp[rp_dst[k] + m * (RP_STRIDE - 1)] = f.rp[k];
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_KFULL + s]);
+            if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
+            return true;
+        };
+
+        Prefetch pa, pb;
+        fetch(0, pa);
+        if (U > 1) fetch(1, pb);
+        for (int u = 0; u < U; u += 2) {
+            if (!step(u, pa)) break;
+            if (u + 2 < U) fetch(u + 2, pa);
+            if (u + 1 >= U) break;
+            if (!step(u + 1, pb)) break;
+            if (u + 3 < U) fetch(u + 3, pb);
         }
         // On an abort, let TMA copies already issued land before the CTA exits.
-        if (*abort_flag && lane == 0) {
-            for (int t = (T > STAGES ? T - STAGES : 0); t < T; ++t)
-                mbar_wait(&bars[B_VFULL + t % STAGES], (t / STAGES) & 1, nullptr, 100000000ull);
+        if (*abort_flag && lw == 0 && lane == 0) {
+            for (int u = (U > S ? U - S : 0); u < U; ++u)
+                mbar_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue
+    } else if (warp == MMA_WARP) {
+        // ---------------------------------------------------------------- MMA issue
         if (lane == 0) {
             const uint32_t idesc_qk = (QK == QK_I8) ? instr_desc(kCS32, kFmtS8, kFmtS8, BM, BN)
                                                     : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
             const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
             const uint32_t sbo_qk = (uint32_t)chunks * 128u;
-            const uint32_t q_base = smem_addr(smem + L.q);
-            const uint32_t p_base = smem_addr(smem + L.p);
-            const uint32_t tm_o = tmem + 256;
-            bool ok = mbar_wait(&bars[B_Q], 0, abort_flag) && mbar_wait(&bars[B_KFULL], 0, abort_flag);
-            auto issue_qk = [&](int buf, int stage) {
-                const uint32_t k_base = smem_addr(smem + (stage ? L.k[1] : L.k[0]));
-                for (int kk = 0; kk < p.dpad / 32; ++kk) {
-                    const uint64_t a = smem_desc(q_base + kk * 256, 128, sbo_qk, kLayoutNone);
-                    const uint64_t b = smem_desc(k_base + kk * 256, 128, sbo_qk, kLayoutNone);
-                    mma_ss<QK>(tmem + buf * 128, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(&bars[B_SFULL + buf]);
-            };
-            if (ok) {
+            bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag);
+            auto issue_qk = [&](int u) -> bool {
+                const int s = u % S, buf = u & 1;
+                if (!mbar_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag)) return false;
+                for (int g = 0; g < NG; ++g)
+                    if (u >= 2 && !mbar_wait(&bars[B_SEMPTY + 2 * g + buf], ((u >> 1) - 1) & 1, abort_flag))
+                        return false;
                 tc_fence_after();
-                issue_qk(0, 0);
-            }
-            for (int t = 0; ok && t < T; ++t) {
-                const int s = t % STAGES;
-                if (t + 1 < T) {
-                    const int s1 = (t + 1) % STAGES, buf = (t + 1) & 1;
-                    ok = mbar_wait(&bars[B_KFULL + s1], ((t + 1) / STAGES) & 1, abort_flag);
-                    if (ok && t + 1 >= 2) ok = mbar_wait(&bars[B_SEMPTY + buf], (((t + 1) >> 1) - 1) & 1, abort_flag);
+                for (int g = 0; g < NG; ++g) {
+                    const uint32_t q_base = smem_addr(smem + L.q + g * L.q_bytes);
+                    const uint32_t k_base = smem_addr(smem + L.k + (s * KVG + (PAIR ? g : 0)) * L.k_bytes);
+                    for (int kk = 0; kk < p.dpad / 32; ++kk)
+                        mma_ss<QK>(tmem + (2 * g + buf) * BN, smem_desc(q_base + kk * 256, 128, sbo_qk, kLayoutNone),
+                                   smem_desc(k_base + kk * 256, 128, sbo_qk, kLayoutNone), idesc_qk,
+                                   kk > 0 ? 1u : 0u);
+                    mma_commit(&bars[B_SFULL + 2 * g + buf]);
+                }
+                return true;
+            };
+            if (ok) ok = issue_qk(0);
+            for (int u = 0; ok && u < U; ++u) {
+                if (u + 1 < U && !(ok = issue_qk(u + 1))) break;
+                if (u >= T) {
+                    const int t = u - T, pb = t & 1, s = u % S;
+                    for (int g = 0; g < NG && ok; ++g)
+                        ok = mbar_wait(&bars[B_PFULL + 2 * g + pb], (t >> 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_qk(buf, s1);
+                    for (int g = 0; g < NG; ++g) {
+                        const uint32_t p_base = smem_addr(smem + L.p + (g * 2 + pb) * BM * BN);
+                        const uint32_t v_base = smem_addr(smem + L.v + (s * KVG + (PAIR ? g : 0)) * L.v_bytes);
+                        for (int kk = 0; kk < BN / 32; ++kk)
+                            mma_ss<QK_I8>(tmem + 256 + 128 * g, smem_desc(p_base + kk * 256, 128, 512, kLayoutNone),
+                                          smem_desc(v_base + kk * 32, 16, 512, kLayoutSw64), idesc_pv,
+                                          (t > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&bars[B_PFREE + 2 * g + pb]);
+                    }
                 }
-                ok = mbar_wait(&bars[B_PFULL], t & 1, abort_flag) &&
-                     mbar_wait(&bars[B_VFULL + s], (t / STAGES) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t v_base = smem_addr(smem + (s ? L.v[1] : L.v[0]));
-                for (int kk = 0; kk < BN / 32; ++kk) {
-                    const uint64_t a = smem_desc(p_base + kk * 256, 128, 1024, kLayoutNone);
-                    const uint64_t b = smem_desc(v_base + kk * 32, 16, 1024, kLayoutSw128);
-                    mma_ss<QK_I8>(tm_o, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars[B_PVDONE]);
-                mma_commit(&bars[B_KVEMPTY + s]);
+                mma_commit(&bars[B_EMPTY + u % S]);
             }
             if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
             // Let every issued MMA finish before TMEM is released.
             mma_commit(&bars[B_FINAL]);
-            if (!mbar_wait(&bars[B_FINAL], 0, abort_flag, 4000000000ull)) atomicOr(p.status, kStatusTimeoutMma);
+            if (!mbar_wait(&bars[B_FINAL], 0, nullptr, 4000000000ull)) atomicOr(p.status, kStatusTimeoutMma);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue
+        // ---------------------------------------------------------------- softmax + epilogue
+        const int g = warp >> 2;                      // row group
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
-        const int r = quarter * 32 + lane;            // row within the tile
+        const int r = quarter * 32 + lane;            // row within the group
+        int bh, q0;
+        bool group_exists;
+        group_coords<PAIR>(p, g, bh, q0, group_exists);
         const int i = q0 + r;
-        const bool row_ok = i < N;
-        const int ie = row_ok ? i : N - 1;
+        const bool row_ok = group_exists && i < N;
+        const int ie = (i < N) ? i : N - 1;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const int kvx = PAIR ? g : 0;
 
-        // Q operand: this thread's row, padding channels zeroed.
+        // Q operand of this row, padding channels zeroed.
         {
-            uint8_t* qop = smem + L.q;
+            uint8_t* qop = smem + L.q + g * L.q_bytes;
             const uint32_t* src = p.bq + ((size_t)bh * N + ie) * W;
             for (int w = 0; w < W; ++w) {
                 const uint32_t bits = row_ok ? __ldg(src + w) : 0u;
@@ -323,140 +572,96 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_Q]);
+            if (lane == 0) mbar_arrive(&bars[B_QREADY]);
         }
         const float cq = row_ok ? __ldg(p.muq + (size_t)bh * N + i) * p.q_scale : 0.f;
-        int rel_base = 0;
-        const float* tab = p.table;
+        const uint64_t cq2 = f2_pack(cq, cq);
+        int rel_base = 0, rp_off = 0;
         if (BIAS == BA_BIAS_RELPOS2D) {
-            const int ri = ie / p.gw, ci = ie - ri * p.gw;
-            rel_base = (ri + p.gh - 1) * (2 * p.gw - 1) + ci + p.gw - 1;
-            tab += (size_t)h * (2 * p.gh - 1) * (2 * p.gw - 1);
+            if (p.relpos_fast) {
+                const int sidx = (BM - 1) - r;             // 127 - (ci - ci0)
+                const int m = sidx & 3;
+                rp_off = (g * 4 + m) * RP_STRIDE + (sidx - m);
+            } else {
+                const int ri = ie / p.gw, ci = ie - ri * p.gw;
+                rel_base = (ri + p.gh - 1) * (2 * p.gw - 1) + ci + p.gw - 1;
+            }
         }
 
-        float m = -INFINITY, l = 0.f;
+        float mrow = -INFINITY;
+        uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        uint64_t neg2 = 0;
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int s = t % STAGES, buf = t & 1;
+        for (int u = 0; u < U; ++u) {
+            const int s = u % S, buf = u & 1;
+            const bool pass_b = u >= T;
+            const int t = pass_b ? u - T : u;
             const int j0 = t * BN;
-            ok = warp_wait(&bars[B_SFULL + buf], (t >> 1) & 1, abort_flag) &&
-                 warp_wait(&bars[B_KFULL + s], (t / STAGES) & 1, abort_flag);
-            if (ok && BIAS == BA_BIAS_DENSE) ok = warp_wait(&bars[B_VFULL + s], (t / STAGES) & 1, abort_flag);
+            const int pb = t & 1;
+            ok = warp_wait(&bars[B_SFULL + 2 * g + buf], (u >> 1) & 1, abort_flag) &&
+                 warp_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag);
+            if (ok && pass_b && t >= 2) ok = warp_wait(&bars[B_PFREE + 2 * g + pb], ((t >> 1) - 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-
-            float sc[BN];
-            {
-                uint32_t z[32];
+            const bool ragged = j0 + BN > N;
+            const float* muk_s = reinterpret_cast<const float*>(smem + L.muk) + (s * KVG + kvx) * BN;
+            const int* koff_s = reinterpret_cast<const int*>(smem + L.koff) + s * BN;
+            const uint8_t* bsm_row = smem + L.b + s * 2 * 16384 + r * 128;
+            const float* rpc = (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast)
+                ? reinterpret_cast<const float*>(smem + L.rp) + (size_t)s * NG * 4 * RP_STRIDE + rp_off : nullptr;
+            const int nvalid = N - j0;
+            uint32_t zr[64];
+            tmem_ld64(tmem + (2 * g + buf) * BN + lane_base, zr);
+            tmem_wait_ld();
+            uint32_t pw[16];
+            float mx[2] = {-INFINITY, -INFINITY};
+            if (!pass_b) {
+                if (ragged)
+                    softmax_tile<QK, BIAS, false, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                                                        nvalid, cq2, neg2, mx, l2, pw);
+                else
+                    softmax_tile<QK, BIAS, false, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                                                         nvalid, cq2, neg2, mx, l2, pw);
+                mrow = fmax3(mrow, mx[0], mx[1]);
+            } else {
+                if (ragged)
+                    softmax_tile<QK, BIAS, true, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                                                       nvalid, cq2, neg2, mx, l2, pw);
+                else
+                    softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                                                        nvalid, cq2, neg2, mx, l2, pw);
+                uint8_t* prow = smem + L.p + (g * 2 + pb) * BM * BN;
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    tmem_ld32(tmem + buf * 128 + c * 32 + lane_base, z);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        sc[c * 32 + e] = (QK == QK_I8) ? __int2float_rn((int)z[e]) : __uint_as_float(z[e]);
-                }
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(prow + core_off(r, c, BN / 16)) =
+                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             }
             tc_fence_before();
+            if (pass_b) fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_SEMPTY + buf]);
-
-            // S = mu_q mu_k z / sqrt(d) + b  (Key design 2), and the tile max
-            const float* muk_s = reinterpret_cast<const float*>(smem + (s ? L.muk[1] : L.muk[0]));
-            const int* koff_s = reinterpret_cast<const int*>(smem + (s ? L.koff[1] : L.koff[0]));
-            const uint8_t* bsm = smem + (s ? L.b[1] : L.b[0]) + r * 128;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c4 = 0; c4 < BN / 4; ++c4) {
-                const float4 mk = *reinterpret_cast<const float4*>(muk_s + 4 * c4);
-                float bb[4] = {0.f, 0.f, 0.f, 0.f};
-                if (BIAS == BA_BIAS_DENSE) {
-                    const int box = c4 >> 3, k = c4 & 7;
-                    const float4 v = *reinterpret_cast<const float4*>(bsm + box * 16384 + ((k ^ (r & 7)) << 4));
-                    bb[0] = v.x; bb[1] = v.y; bb[2] = v.z; bb[3] = v.w;
-                } else if (BIAS == BA_BIAS_RELPOS2D) {
-                    const int4 ko = *reinterpret_cast<const int4*>(koff_s + 4 * c4);
-                    bb[0] = __ldg(tab + rel_base - ko.x);
-                    bb[1] = __ldg(tab + rel_base - ko.y);
-                    bb[2] = __ldg(tab + rel_base - ko.z);
-                    bb[3] = __ldg(tab + rel_base - ko.w);
-                }
-                const float mkv[4] = {mk.x, mk.y, mk.z, mk.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = 4 * c4 + e;
-                    const float x = fmaf(sc[c] * mkv[e], cq, bb[e]);
-                    sc[c] = x;
-                    mx = fmaxf(mx, x);
-                }
+            if (lane == 0) {
+                mbar_arrive(&bars[B_SEMPTY + 2 * g + buf]);
+                mbar_arrive(&bars[B_EMPTY + s]);
+                if (pass_b) mbar_arrive(&bars[B_PFULL + 2 * g + pb]);
             }
-            if (j0 + BN > N) {               // ragged last tile: keys >= N do not exist
-                mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    if (j0 + c >= N) sc[c] = -INFINITY;
-                    mx = fmaxf(mx, sc[c]);
-                }
-            }
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2((m - m_new) * LOG2E);      // 0 on the first tile
-            const float neg = -m_new * LOG2E;
-            l *= alpha;
-
-            // P buffer and accumulator are free once PV of the previous tile is done.
-            if (t > 0 && !warp_wait(&bars[B_PVDONE], (t - 1) & 1, abort_flag)) { ok = false; break; }
-            if (t > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
-                tc_fence_after();
-                const long long aq = (long long)__float2uint_rn(alpha * 2147483648.0f);
-                for (int c = 0; c < p.dv; c += 16) {
-                    uint32_t acc[16];
-                    tmem_ld16(tmem + 256 + c + lane_base, acc);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        acc[e] = (uint32_t)(int)(((long long)(int)acc[e] * aq + (1ll << 30)) >> 31);
-                    tmem_st16(tmem + 256 + c + lane_base, acc);
-                }
-                tmem_wait_st();
-            }
-
-            // P~ = exp(S - m), l += P~, pq = round(255 P~) as u8 (Key design 3)
-            uint8_t* prow = smem + L.p + (r >> 3) * 1024 + (r & 7) * 16;
-#pragma unroll
-            for (int kc = 0; kc < BN / 16; ++kc) {
-                uint32_t wv[4];
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint32_t b4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float pr = ex2(fmaf(sc[kc * 16 + g * 4 + e], LOG2E, neg));
-                        l += pr;
-                        b4[e] = __float_as_uint(fmaf(pr, 255.f, 12582912.f));   // low byte = rint(255 P~)
-                    }
-                    wv[g] = __byte_perm(__byte_perm(b4[0], b4[1], 0x0040), __byte_perm(b4[2], b4[3], 0x0040), 0x5410);
-                }
-                *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_PFULL]);
-            m = m_new;
+            if (u == T - 1) neg2 = f2_pack(-mrow * LOG2E, -mrow * LOG2E);
         }
 
         // Epilogue: O = sv * acc / (255 l).
-        if (ok) ok = warp_wait(&bars[B_PVDONE], (T - 1) & 1, abort_flag);
+        if (ok) ok = warp_wait(&bars[B_PFREE + 2 * g + ((T - 1) & 1)], ((T - 1) >> 1) & 1, abort_flag);
         if (!ok) {
             if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutSoftmax);
         } else {
             tc_fence_after();
-            const float inv = 1.f / (255.f * l);
+            float la, lb, lc, ld;
+            f2_unpack(l2[0], la, lb);
+            f2_unpack(l2[1], lc, ld);
+            const float inv = 1.f / (255.f * ((la + lb) + (lc + ld)));
             OutT* dst = static_cast<OutT*>(p.out) + ((size_t)bh * N + ie) * p.d;
             const float* svp = p.sv + (size_t)bh * p.d;
             for (int c = 0; c < p.dv; c += 16) {
                 uint32_t acc[16];
-                tmem_ld16(tmem + 256 + c + lane_base, acc);
+                tmem_ld16(tmem + 256 + 128 * g + c + lane_base, acc);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -469,7 +674,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -493,31 +698,42 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 int dv_of(int d) { return (d + 15) / 16 * 16; }
 
-size_t smem_bytes(int d, int bias_kind)
+constexpr size_t kSmemLimit = 227u * 1024u;
+
+size_t smem_bytes(int d, int bias_kind, int stages)
 {
-    const Layout L = make_layout(32 * words_for(d), dv_of(d), bias_kind == BA_BIAS_DENSE);
+    const Layout L = make_layout(32 * words_for(d), dv_of(d), bias_kind, stages);
     return (size_t)L.total + 1024;   // slack for the manual 1 KB alignment
 }
 
+// Deepest pipeline (2..4 stages) that fits; 0 if even 2 do not.
+int pick_stages(int d, int bias_kind)
+{
+    for (int s = MAX_STAGES; s >= 2; --s)
+        if (smem_bytes(d, bias_kind, s) <= kSmemLimit) return s;
+    return 0;
+}
+
 template <int QK, typename OutT, int BIAS>
-cudaError_t launch_t(const CUtensorMap& tv, const CUtensorMap& tb, const Params& p, int BH, size_t smem,
-                     cudaStream_t st)
+cudaError_t launch_t(const CUtensorMap& tv, const CUtensorMap& tb, const Params& p, size_t smem, cudaStream_t st)
 {
     auto kern = attn_tc_kernel<QK, OutT, BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(p.N, BM), BH);
+    dim3 grid = (BIAS == BA_BIAS_DENSE)
+                    ? dim3(ceil_div(p.N, BM), p.H, ceil_div(p.B, 2))
+                    : dim3(ceil_div(p.N, BM * NG), p.B * p.H, 1);
     kern<<<grid, NUM_THREADS, smem, st>>>(tv, tb, p);
     return cudaGetLastError();
 }
 
 template <int QK, typename OutT>
-cudaError_t launch_bias(int kind, const CUtensorMap& tv, const CUtensorMap& tb, const Params& p, int BH,
-                        size_t smem, cudaStream_t st)
+cudaError_t launch_bias(int kind, const CUtensorMap& tv, const CUtensorMap& tb, const Params& p, size_t smem,
+                        cudaStream_t st)
 {
-    if (kind == BA_BIAS_DENSE) return launch_t<QK, OutT, BA_BIAS_DENSE>(tv, tb, p, BH, smem, st);
-    if (kind == BA_BIAS_RELPOS2D) return launch_t<QK, OutT, BA_BIAS_RELPOS2D>(tv, tb, p, BH, smem, st);
-    return launch_t<QK, OutT, BA_BIAS_NONE>(tv, tb, p, BH, smem, st);
+    if (kind == BA_BIAS_DENSE) return launch_t<QK, OutT, BA_BIAS_DENSE>(tv, tb, p, smem, st);
+    if (kind == BA_BIAS_RELPOS2D) return launch_t<QK, OutT, BA_BIAS_RELPOS2D>(tv, tb, p, smem, st);
+    return launch_t<QK, OutT, BA_BIAS_NONE>(tv, tb, p, smem, st);
 }
 
 }  // namespace
@@ -526,9 +742,7 @@ bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d)
 {
     (void)gh; (void)gw; (void)N;
     if (d < 1 || d > 128) return false;
-    // The whole pipeline must fit one CTA's shared memory, with room to keep a
-    // second CTA off the SM (it would only wait for tensor memory).
-    return smem_bytes(d, bias_kind) <= 227u * 1024u;
+    return pick_stages(d, bias_kind) >= 2;
 }
 
 cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
@@ -552,7 +766,7 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
         cuuint32_t box[3] = {(cuuint32_t)BN, (cuuint32_t)dv, 1};
         cuuint32_t es[3] = {1, 1, 1};
         if (encode(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(vq), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
@@ -571,23 +785,25 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     p.bq = bq; p.muq = muq; p.bk = bk; p.muk = muk; p.sv = sv;
     p.table = bias_kind == BA_BIAS_RELPOS2D ? bias : nullptr;
     p.out = out;
-    p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
+    p.B = B; p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
     p.n_tiles = ceil_div(N, BN);
+    p.stages = pick_stages(d, bias_kind);
     p.gh = gh; p.gw = gw;
+    // A 128-row query tile and a 64-key tile then each lie inside one grid row.
+    p.relpos_fast = (bias_kind == BA_BIAS_RELPOS2D && gw % BM == 0) ? 1 : 0;
     p.q_scale = (float)(1.0 / sqrt((double)d));
     p.status = status;
 
-    // Ask for enough shared memory that only one CTA fits on an SM: each CTA
-    // takes all 512 TMEM columns.
-    size_t smem = smem_bytes(d, bias_kind);
+    // One CTA per SM: each takes all 512 TMEM columns.
+    size_t smem = smem_bytes(d, bias_kind, p.stages);
     if (smem < 120u * 1024u) smem = 120u * 1024u;
 
-    const bool f8 = variant == BA_QK_TC_F8;
+    const bool f8 = variant != BA_QK_TC_I8;
     if (out_dt == BA_BF16)
-        return f8 ? launch_bias<QK_F8, __nv_bfloat16>(bias_kind, tv, tb, p, BH, smem, st)
-                  : launch_bias<QK_I8, __nv_bfloat16>(bias_kind, tv, tb, p, BH, smem, st);
-    return f8 ? launch_bias<QK_F8, float>(bias_kind, tv, tb, p, BH, smem, st)
-              : launch_bias<QK_I8, float>(bias_kind, tv, tb, p, BH, smem, st);
+        return f8 ? launch_bias<QK_F8, __nv_bfloat16>(bias_kind, tv, tb, p, smem, st)
+                  : launch_bias<QK_I8, __nv_bfloat16>(bias_kind, tv, tb, p, smem, st);
+    return f8 ? launch_bias<QK_F8, float>(bias_kind, tv, tb, p, smem, st)
+              : launch_bias<QK_I8, float>(bias_kind, tv, tb, p, smem, st);
 }
 
 }  // namespace ba

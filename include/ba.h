@@ -98,7 +98,7 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
  * KD1-KD3 + FW -- the fused forward.  For every (b, h, i):
  *   z_ij  = s_i . t_j = d - 2 popcount(bq_i XOR bk_j)                   (KD1)
  *   S_ij  = muq_i muk_j z_ij / sqrt(d) + b_ij                            (KD2)
- *   P~_ij = exp(S_ij - m_i) with m_i the running row maximum (FW),
+ *   P~_ij = exp(S_ij - m_i) with m_i = max_j S_ij, the exact row maximum,
  *   pq_ij = round(255 P~_ij) in 0..255, l_i = sum_j P~_ij (unquantised)  (KD3)
  *   O_ic  = sv_c * sum_j pq_ij vq_jc / (255 l_i)                         (KD3)
  * Inputs: bq, bk [B, H, N, W] from ba_pack_qk; muq, muk [B, H, N];
@@ -109,8 +109,9 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
  *   grid_h * grid_w, and b_ij = table[h][(ri - rj + grid_h - 1) *
  *   (2 grid_w - 1) + (ci - cj + grid_w - 1)].
  * out: [B, H, N, d] in out_dt (BA_F32 or BA_BF16).
- * The running maximum means pq may differ from an exact-maximum quantisation
- * by one unit; the result stays within the stated parity tolerance.
+ * The keys are swept twice inside the kernel (maximum first, then P and PV),
+ * so pq is quantised against the exact maximum rather than a running one;
+ * fp32 arithmetic can still move a code sitting on a rounding boundary by one.
  */
 ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
                            const uint32_t* bk, const float* muk,
