@@ -24,8 +24,9 @@
 //     memory (kind::i8 -> s32, or kind::f8f6f4 with e4m3 +-1 -> f32; both are
 //     exact), into double-buffered S tiles in TMEM, so the next tile's QK
 //     overlaps this tile's softmax;
-//   * PV runs on tcgen05.mma kind::i8 (u8 P from shared memory, s8 V tiles
-//     brought in by TMA), accumulating in TMEM across all key tiles;
+//   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (the
+//     softmax writes it over the S tile it came from) and s8 V tiles brought
+//     in by TMA, accumulating in TMEM across all key tiles;
 //   * the softmax pulls each 64-key S tile out of TMEM with one load and does
 //     its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with a 3-input
 //     max;
@@ -59,19 +60,31 @@ constexpr int NG = 2;                   // row groups per CTA
 constexpr int BN = 64;                  // keys per tile
 constexpr int MAX_STAGES = 4;
 constexpr int NUM_SOFTMAX_WARPS = 4 * NG;
-constexpr int NUM_LOAD_WARPS = 4;
+constexpr int NUM_LOAD_WARPS = 3;
 constexpr int NUM_LOADERS = 32 * NUM_LOAD_WARPS;
 constexpr int LOAD_WARP0 = NUM_SOFTMAX_WARPS;               // 8
 constexpr int MMA_WARP = LOAD_WARP0 + NUM_LOAD_WARPS;       // 12
-constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 416
+constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 384
+// Warps are given registers in groups of four: 12 warps leave 168 per thread.
+constexpr int MAX_REGS = 168;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int QK_I8 = 0, QK_F8 = 1;
+// Bias variants of the kernel: the three of the ABI, plus a rel-pos fast path
+// for grid widths that are multiples of 128 (tiles then sit inside one grid row).
+constexpr int BIAS_RP_FAST = 3;
+__host__ __device__ constexpr bool is_relpos(int b) { return b == BA_BIAS_RELPOS2D || b == BIAS_RP_FAST; }
 constexpr int RP_SPAN = BM + BN - 2;    // largest offset inside a rel-pos window (190)
 constexpr int RP_VALS = RP_SPAN + 1;    // values in a window
 constexpr int RP_WIN = 192;             // entries per shifted copy of a window (RP_STRIDE >= RP_WIN)
 constexpr int RP_STRIDE = 200;          // floats between copies (8 words mod 32: conflict-free)
-constexpr int RP_PER_THREAD = (NG * RP_VALS + NUM_LOADERS - 1) / NUM_LOADERS;   // 3
+// Each loader thread builds four consecutive entries of all four copies of
+// one window: it needs seven consecutive window values.
+constexpr int RP_BLOCKS = NG * RP_WIN / 4;                                       // 96
+constexpr int RP_PER_THREAD = 7;
+static_assert(RP_BLOCKS <= NUM_LOADERS, "one rel-pos block per loader thread");
+constexpr int K_PER_THREAD = (2 * BN * 4 + NUM_LOADERS - 1) / NUM_LOADERS;       // sign words, <= 6
+constexpr int MU_PER_THREAD = (2 * BN + NUM_LOADERS - 1) / NUM_LOADERS;          // key scales, <= 2
 
 // Barrier slots.
 enum {
@@ -79,10 +92,9 @@ enum {
     B_FULL = 1,                      // [stage] operands, scales, bias (and V in pass B) ready
     B_EMPTY = B_FULL + MAX_STAGES,   // [stage] stage may be overwritten
     B_SFULL = B_EMPTY + MAX_STAGES,  // [NG][2] S tile in TMEM ready
-    B_SEMPTY = B_SFULL + 2 * NG,     // [NG][2] softmax done with S buffer
-    B_PFULL = B_SEMPTY + 2 * NG,     // [NG][2] u8 P tile written
-    B_PFREE = B_PFULL + 2 * NG,      // [NG][2] PV that read P buffer finished
-    B_FINAL = B_PFREE + 2 * NG,
+    B_SDONE = B_SFULL + 2 * NG,      // [NG][2] softmax done with the S buffer (pass B: u8 P written into it)
+    B_OREADY = B_SDONE + 2 * NG,     // every PV finished
+    B_FINAL = B_OREADY + 1,
     NUM_BARS
 };
 
@@ -92,7 +104,6 @@ struct Layout {
     uint32_t b;                 // [stage][2] dense bias boxes, 16 KB each (SW128)
     uint32_t q, q_bytes;        // [NG] Q operands
     uint32_t k, k_bytes;        // [stage][kvg] K operands
-    uint32_t p;                 // [NG][2] P tiles, 8 KB each
     uint32_t muk, koff;         // [stage][kvg][BN], [stage][BN]
     uint32_t rp;                // [stage][NG][4][RP_STRIDE] rel-pos windows
     uint32_t bars, misc, total;
@@ -113,10 +124,9 @@ __host__ __device__ inline Layout make_layout(int dpad, int dv, int bias_kind, i
     L.q = off; off += NG * L.q_bytes;
     L.k_bytes = align_up((uint32_t)BN * dpad, 1024);
     L.k = off; off += stages * L.kvg * L.k_bytes;
-    L.p = off; off += NG * 2 * BM * BN;
     L.muk = off; off += stages * L.kvg * BN * 4;
-    L.koff = off; off += stages * BN * 4;
-    L.rp = off; off += (bias_kind == BA_BIAS_RELPOS2D) ? stages * NG * 4 * RP_STRIDE * 4u : 0u;
+    L.koff = off; off += (bias_kind == BA_BIAS_RELPOS2D) ? stages * BN * 4 : 0u;
+    L.rp = off; off += (bias_kind == BIAS_RP_FAST) ? stages * NG * 4 * RP_STRIDE * 4u : 0u;
     L.bars = off; off += NUM_BARS * 8;
     L.misc = off; off += 16;            // TMEM base address, abort flag
     L.total = off;
@@ -132,7 +142,7 @@ struct Params {
     const float* table;      // 2-D relative-position table (global)
     void* out;
     int B, H, N, d, W, dpad, dv, n_tiles, stages;
-    int gh, gw, relpos_fast;
+    int gh, gw;
     float q_scale;           // 1 / sqrt(d)
     unsigned* status;
 };
@@ -221,21 +231,30 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
     const uint64_t L2E = f2_pack(LOG2E, LOG2E);
     const uint64_t C255 = f2_pack(255.f, 255.f);
     const uint64_t MAGIC = f2_pack(12582912.f, 12582912.f);
-#pragma unroll
-    for (int k4 = 0; k4 < BN / 4; ++k4) {
-        const float4 mk = *reinterpret_cast<const float4*>(mks + 4 * k4);
-        float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+    // The key scales and bias values come from shared memory; they are
+    // fetched PF groups of four keys ahead so their latency overlaps math.
+    constexpr int PF = 3;
+    auto fetch = [&](int k4, float4& mk, float4& bb) {
+        mk = *reinterpret_cast<const float4*>(mks + 4 * k4);
+        bb = make_float4(0.f, 0.f, 0.f, 0.f);
         if (BIAS == BA_BIAS_DENSE) {
             bb = *reinterpret_cast<const float4*>(bsm_row + (k4 >> 3) * 16384 + (((k4 & 7) ^ bsm_sw) << 4));
+        } else if (BIAS == BIAS_RP_FAST) {
+            bb = *reinterpret_cast<const float4*>(rp_copy + 4 * k4);
         } else if (BIAS == BA_BIAS_RELPOS2D) {
-            if (rp_copy) {
-                bb = *reinterpret_cast<const float4*>(rp_copy + 4 * k4);
-            } else {
-                const int4 ko = *reinterpret_cast<const int4*>(koff + 4 * k4);
-                bb = make_float4(__ldg(tab_h + rel_base - ko.x), __ldg(tab_h + rel_base - ko.y),
-                                 __ldg(tab_h + rel_base - ko.z), __ldg(tab_h + rel_base - ko.w));
-            }
+            const int4 ko = *reinterpret_cast<const int4*>(koff + 4 * k4);
+            bb = make_float4(__ldg(tab_h + rel_base - ko.x), __ldg(tab_h + rel_base - ko.y),
+                             __ldg(tab_h + rel_base - ko.z), __ldg(tab_h + rel_base - ko.w));
         }
+    };
+    float4 mkq[PF], bbq[PF];
+#pragma unroll
+    for (int k = 0; k < PF; ++k) fetch(k, mkq[k], bbq[k]);
+#pragma unroll
+    for (int k4 = 0; k4 < BN / 4; ++k4) {
+        const float4 mk = mkq[k4 % PF];
+        const float4 bb = bbq[k4 % PF];
+        if (k4 + PF < BN / 4) fetch(k4 + PF, mkq[k4 % PF], bbq[k4 % PF]);
         uint64_t z01, z23;
         if (QK == QK_F8) {
             z01 = f2_pack(__uint_as_float(zr[4 * k4]), __uint_as_float(zr[4 * k4 + 1]));
@@ -286,14 +305,14 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
 // What one loader thread fetches from global memory for one step, held in
 // registers until the stage is free.
 struct Prefetch {
-    uint32_t kbits[4];           // sign words for up to 4 (key, word) items
-    float muk;                   // one key scale
-    int koff;                    // one key's rel-pos offset (general rel-pos path)
-    float rp[RP_PER_THREAD];     // rel-pos window values
+    uint32_t kbits[K_PER_THREAD];   // sign words of this thread's (key, word) items
+    float muk[MU_PER_THREAD];       // key scales
+    int koff[MU_PER_THREAD];        // keys' rel-pos offsets (general rel-pos path)
+    float rp[RP_PER_THREAD];        // seven consecutive reversed-window values
 };
 
 template <int QK, typename OutT, int BIAS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __maxnreg__(MAX_REGS)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
                const Params p)
 {
@@ -312,7 +331,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     const int S = p.stages;
     const int chunks = p.dpad / 16;
     const int h = PAIR ? (int)blockIdx.y : (int)(blockIdx.y % p.H);
-    const float* tab_h = (BIAS == BA_BIAS_RELPOS2D)
+    const float* tab_h = is_relpos(BIAS)
                              ? p.table + (size_t)h * (2 * p.gh - 1) * (2 * p.gw - 1) : nullptr;
 
     if (threadIdx.x == 0) {
@@ -323,10 +342,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
         }
         for (int b = 0; b < 2 * NG; ++b) {
             mbar_init(&bars[B_SFULL + b], 1);
-            mbar_init(&bars[B_SEMPTY + b], 4);
-            mbar_init(&bars[B_PFULL + b], 4);
-            mbar_init(&bars[B_PFREE + b], 1);
+            mbar_init(&bars[B_SDONE + b], 4);
         }
+        mbar_init(&bars[B_OREADY], 1);
         mbar_init(&bars[B_FINAL], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -363,11 +381,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             if (KVG > 1) group_coords<PAIR>(p, 1, kvbh1, q0x, ex);
         }
         const int kitems = KVG * BN * W;
-        const uint32_t* kbase[4];
-        int krow[4];
-        uint32_t kdst[4];
+        const uint32_t* kbase[K_PER_THREAD];
+        int krow[K_PER_THREAD];
+        uint32_t kdst[K_PER_THREAD];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < K_PER_THREAD; ++k) {
             const int e = ltid + k * NUM_LOADERS;
             const int x = e / (BN * W), rem = e - x * (BN * W);
             const int r = rem / W, w = rem - r * W;
@@ -375,52 +393,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             kbase[k] = p.bk + ((size_t)(x ? kvbh1 : kvbh0) * N + r) * W + w;
             kdst[k] = (uint32_t)(x * L.k_bytes) + core_off(r, 2 * w, chunks);
         }
-        const bool has_mu = ltid < KVG * BN;
-        const int mu_row = ltid % BN;
-        const float* mu_base = p.muk + (size_t)((ltid / BN) ? kvbh1 : kvbh0) * N + mu_row;
-        const float* rp_src[RP_PER_THREAD];
-        int rp_dst[RP_PER_THREAD], rp_v[RP_PER_THREAD];
+        int mu_row[MU_PER_THREAD];
+        const float* mu_base[MU_PER_THREAD];
 #pragma unroll
-        for (int k = 0; k < RP_PER_THREAD; ++k) {
+        for (int k = 0; k < MU_PER_THREAD; ++k) {
             const int e = ltid + k * NUM_LOADERS;
-            rp_v[k] = -1;
-            rp_src[k] = tab_h;
-            rp_dst[k] = 0;
-            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast && e < NG * RP_VALS) {
-                const int g = e / RP_VALS, v = e - g * RP_VALS;
-                int bhg, q0g;
-                bool ex;
-                group_coords<PAIR>(p, g, bhg, q0g, ex);
-                if (q0g >= N) q0g = N - BM;              // an empty group still reads inside the table
-                const int ri = q0g / p.gw, ci0 = q0g - ri * p.gw;
-                // Rr[v] = R[xlo + RP_SPAN - v] with R the table row of offset
-                // ri - rj and xlo = ci0 - cj0 - (BN - 1) + gw - 1; only the
-                // key-tile part rj * (2 gw - 1) + cj0 changes per step.
-                rp_src[k] = tab_h + (ptrdiff_t)(ri + p.gh - 1) * (2 * p.gw - 1) + ci0 - (BN - 1) + p.gw - 1 + RP_SPAN - v;
-                rp_v[k] = v;
-                rp_dst[k] = g * 4 * RP_STRIDE + v;
-            }
+            mu_row[k] = (e < KVG * BN) ? e % BN : (1 << 30);   // never valid
+            mu_base[k] = p.muk + (size_t)((e / BN) ? kvbh1 : kvbh0) * N + e % BN;
+        }
+        // Rel-pos window block of this thread: group rp_g, entries rp_y..rp_y+3
+        // of each copy, built from Rr[rp_y .. rp_y + 6] (Rr = reversed window).
+        const float* rp_src = tab_h;
+        int rp_y = -1, rp_g = 0;
+        if (BIAS == BIAS_RP_FAST && ltid < RP_BLOCKS) {
+            rp_g = ltid / (RP_WIN / 4);
+            rp_y = (ltid - rp_g * (RP_WIN / 4)) * 4;
+            int bhg, q0g;
+            bool ex;
+            group_coords<PAIR>(p, rp_g, bhg, q0g, ex);
+            if (q0g >= N) q0g = N - BM;              // an empty group still reads inside the table
+            const int ri = q0g / p.gw, ci0 = q0g - ri * p.gw;
+            // Rr[v] = R[xlo + RP_SPAN - v] with R the table row of offset ri - rj
+            // and xlo = ci0 - cj0 - (BN - 1) + gw - 1; only the key-tile part
+            // rj * (2 gw - 1) + cj0 changes per step.
+            rp_src = tab_h + (ptrdiff_t)(ri + p.gh - 1) * (2 * p.gw - 1) + ci0 - (BN - 1) + p.gw - 1 + RP_SPAN - rp_y;
         }
 
         auto fetch = [&](int u, Prefetch& f) {
             const int t = (u >= T) ? u - T : u;
             const int j0 = t * BN;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < K_PER_THREAD; ++k)
                 f.kbits[k] = (j0 + krow[k] < N) ? __ldg(kbase[k] + (size_t)j0 * W) : 0u;
-            f.muk = (has_mu && j0 + mu_row < N) ? __ldg(mu_base + j0) : 0.f;
-            f.koff = 0;
-            if (BIAS == BA_BIAS_RELPOS2D && !p.relpos_fast && ltid < BN) {
-                const int jj = min(j0 + ltid, N - 1);
-                const int rj = jj / p.gw, cj = jj - rj * p.gw;
-                f.koff = rj * (2 * p.gw - 1) + cj;
+#pragma unroll
+            for (int k = 0; k < MU_PER_THREAD; ++k) {
+                f.muk[k] = (j0 + mu_row[k] < N) ? __ldg(mu_base[k] + j0) : 0.f;
+                f.koff[k] = 0;
+                const int e = ltid + k * NUM_LOADERS;
+                if (BIAS == BA_BIAS_RELPOS2D && e < BN) {
+                    const int jj = min(j0 + e, N - 1);
+                    const int rj = jj / p.gw, cj = jj - rj * p.gw;
+                    f.koff[k] = rj * (2 * p.gw - 1) + cj;
+                }
             }
-            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast) {
+            if (BIAS == BIAS_RP_FAST) {
                 const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
                 const ptrdiff_t shift = (ptrdiff_t)rj * (2 * p.gw - 1) + cj0;
 #pragma unroll
                 for (int k = 0; k < RP_PER_THREAD; ++k)
-                    f.rp[k] = (rp_v[k] >= 0) ? __ldg(rp_src[k] - shift) : 0.f;
+                    f.rp[k] = (rp_y >= 0 && rp_y + k <= RP_SPAN) ? __ldg(rp_src - shift - k) : 0.f;
             }
         };
 
@@ -449,25 +470,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             }
             uint8_t* kop = smem + L.k + s * KVG * L.k_bytes;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < K_PER_THREAD; ++k) {
                 if (krow[k] < BN) {
                     *reinterpret_cast<uint4*>(kop + kdst[k]) = expand16<QK>(f.kbits[k] & 0xFFFFu, 0xFFFFu);
                     *reinterpret_cast<uint4*>(kop + kdst[k] + 128) = expand16<QK>(f.kbits[k] >> 16, 0xFFFFu);
                 }
             }
-            if (has_mu) {
-                reinterpret_cast<float*>(smem + L.muk)[s * KVG * BN + ltid] = f.muk;
-                if (BIAS == BA_BIAS_RELPOS2D && !p.relpos_fast && ltid < BN)
-                    reinterpret_cast<int*>(smem + L.koff)[s * BN + ltid] = f.koff;
-            }
-            if (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast) {
-                // Copy m of group g holds Rr[y + m]: value Rr[v] goes to y = v - m.
-                float* rp = reinterpret_cast<float*>(smem + L.rp) + (size_t)s * NG * 4 * RP_STRIDE;
 #pragma unroll
-                for (int k = 0; k < RP_PER_THREAD; ++k) {
+            for (int k = 0; k < MU_PER_THREAD; ++k) {
+                const int e = ltid + k * NUM_LOADERS;
+                if (e < KVG * BN) {
+                    reinterpret_cast<float*>(smem + L.muk)[s * KVG * BN + e] = f.muk[k];
+                    if (BIAS == BA_BIAS_RELPOS2D && e < BN)
+                        reinterpret_cast<int*>(smem + L.koff)[s * BN + e] = f.koff[k];
+                }
+            }
+            if (BIAS == BIAS_RP_FAST) {
+                // Copy m of group g holds Rr[y + m] at entry y.
+                if (rp_y >= 0) {
+                    float* dst = reinterpret_cast<float*>(smem + L.rp) + ((size_t)s * NG * 4 + rp_g * 4) * RP_STRIDE + rp_y;
 #pragma unroll
                     for (int m = 0; m < 4; ++m)
-                        if (rp_v[k] >= m) rp[rp_dst[k] + m * (RP_STRIDE - 1)] = f.rp[k];
+                        *reinterpret_cast<float4*>(dst + m * RP_STRIDE) =
+                            make_float4(f.rp[m], f.rp[m + 1], f.rp[m + 2], f.rp[m + 3]);
                 }
             }
             fence_proxy_async_smem();
@@ -500,20 +525,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
             const uint32_t sbo_qk = (uint32_t)chunks * 128u;
             bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag);
+            // Descriptors are built once; moving along a buffer only adds to the
+            // start-address field (bytes / 16), which never carries out.
+            const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
+            const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
+            const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
+            const uint32_t q_step = L.q_bytes >> 4, k_step = L.k_bytes >> 4, v_step = L.v_bytes >> 4;
+            const int kq = p.dpad / 32;
             auto issue_qk = [&](int u) -> bool {
                 const int s = u % S, buf = u & 1;
                 if (!mbar_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag)) return false;
                 for (int g = 0; g < NG; ++g)
-                    if (u >= 2 && !mbar_wait(&bars[B_SEMPTY + 2 * g + buf], ((u >> 1) - 1) & 1, abort_flag))
+                    if (u >= 2 && !mbar_wait(&bars[B_SDONE + 2 * g + buf], ((u >> 1) - 1) & 1, abort_flag))
                         return false;
                 tc_fence_after();
                 for (int g = 0; g < NG; ++g) {
-                    const uint32_t q_base = smem_addr(smem + L.q + g * L.q_bytes);
-                    const uint32_t k_base = smem_addr(smem + L.k + (s * KVG + (PAIR ? g : 0)) * L.k_bytes);
-                    for (int kk = 0; kk < p.dpad / 32; ++kk)
-                        mma_ss<QK>(tmem + (2 * g + buf) * BN, smem_desc(q_base + kk * 256, 128, sbo_qk, kLayoutNone),
-                                   smem_desc(k_base + kk * 256, 128, sbo_qk, kLayoutNone), idesc_qk,
-                                   kk > 0 ? 1u : 0u);
+                    const uint64_t dq = dq0 + g * q_step;
+                    const uint64_t dk = dk0 + (s * KVG + (PAIR ? g : 0)) * k_step;
+                    const uint32_t d_tmem = tmem + (2 * g + buf) * BN;
+                    for (int kk = 0; kk < kq; ++kk)
+                        mma_ss<QK>(d_tmem, dq + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
                     mma_commit(&bars[B_SFULL + 2 * g + buf]);
                 }
                 return true;
@@ -522,23 +553,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             for (int u = 0; ok && u < U; ++u) {
                 if (u + 1 < U && !(ok = issue_qk(u + 1))) break;
                 if (u >= T) {
-                    const int t = u - T, pb = t & 1, s = u % S;
+                    // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
+                    const int t = u - T, buf = u & 1, s = u % S;
                     for (int g = 0; g < NG && ok; ++g)
-                        ok = mbar_wait(&bars[B_PFULL + 2 * g + pb], (t >> 1) & 1, abort_flag);
+                        ok = mbar_wait(&bars[B_SDONE + 2 * g + buf], (u >> 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     for (int g = 0; g < NG; ++g) {
-                        const uint32_t p_base = smem_addr(smem + L.p + (g * 2 + pb) * BM * BN);
-                        const uint32_t v_base = smem_addr(smem + L.v + (s * KVG + (PAIR ? g : 0)) * L.v_bytes);
+                        const uint64_t dv = dv0 + (s * KVG + (PAIR ? g : 0)) * v_step;
+                        const uint32_t a_tmem = tmem + (2 * g + buf) * BN;
                         for (int kk = 0; kk < BN / 32; ++kk)
-                            mma_ss<QK_I8>(tmem + 256 + 128 * g, smem_desc(p_base + kk * 256, 128, 512, kLayoutNone),
-                                          smem_desc(v_base + kk * 32, 16, 512, kLayoutSw64), idesc_pv,
-                                          (t > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&bars[B_PFREE + 2 * g + pb]);
+                            mma_ts_i8(tmem + 256 + 128 * g, a_tmem + kk * 8, dv + kk * 2, idesc_pv,
+                                      (t > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(&bars[B_EMPTY + u % S]);
             }
+            if (ok) mma_commit(&bars[B_OREADY]);
             if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
             // Let every issued MMA finish before TMEM is released.
             mma_commit(&bars[B_FINAL]);
@@ -577,8 +608,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
         const float cq = row_ok ? __ldg(p.muq + (size_t)bh * N + i) * p.q_scale : 0.f;
         const uint64_t cq2 = f2_pack(cq, cq);
         int rel_base = 0, rp_off = 0;
-        if (BIAS == BA_BIAS_RELPOS2D) {
-            if (p.relpos_fast) {
+        if (is_relpos(BIAS)) {
+            if (BIAS == BIAS_RP_FAST) {
                 const int sidx = (BM - 1) - r;             // 127 - (ci - ci0)
                 const int m = sidx & 3;
                 rp_off = (g * 4 + m) * RP_STRIDE + (sidx - m);
@@ -597,17 +628,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             const bool pass_b = u >= T;
             const int t = pass_b ? u - T : u;
             const int j0 = t * BN;
-            const int pb = t & 1;
             ok = warp_wait(&bars[B_SFULL + 2 * g + buf], (u >> 1) & 1, abort_flag) &&
                  warp_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag);
-            if (ok && pass_b && t >= 2) ok = warp_wait(&bars[B_PFREE + 2 * g + pb], ((t >> 1) - 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const bool ragged = j0 + BN > N;
             const float* muk_s = reinterpret_cast<const float*>(smem + L.muk) + (s * KVG + kvx) * BN;
             const int* koff_s = reinterpret_cast<const int*>(smem + L.koff) + s * BN;
             const uint8_t* bsm_row = smem + L.b + s * 2 * 16384 + r * 128;
-            const float* rpc = (BIAS == BA_BIAS_RELPOS2D && p.relpos_fast)
+            const float* rpc = (BIAS == BIAS_RP_FAST)
                 ? reinterpret_cast<const float*>(smem + L.rp) + (size_t)s * NG * 4 * RP_STRIDE + rp_off : nullptr;
             const int nvalid = N - j0;
             uint32_t zr[64];
@@ -630,25 +659,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 else
                     softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                         nvalid, cq2, neg2, mx, l2, pw);
-                uint8_t* prow = smem + L.p + (g * 2 + pb) * BM * BN;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(prow + core_off(r, c, BN / 16)) =
-                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                // The u8 codes go back into this row's lane of the S buffer: the
+                // PV product reads them from TMEM.
+                tmem_st16(tmem + (2 * g + buf) * BN + lane_base, pw);
+                tmem_wait_st();
             }
             tc_fence_before();
-            if (pass_b) fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars[B_SEMPTY + 2 * g + buf]);
+                mbar_arrive(&bars[B_SDONE + 2 * g + buf]);
                 mbar_arrive(&bars[B_EMPTY + s]);
-                if (pass_b) mbar_arrive(&bars[B_PFULL + 2 * g + pb]);
             }
             if (u == T - 1) neg2 = f2_pack(-mrow * LOG2E, -mrow * LOG2E);
         }
 
         // Epilogue: O = sv * acc / (255 l).
-        if (ok) ok = warp_wait(&bars[B_PFREE + 2 * g + ((T - 1) & 1)], ((T - 1) >> 1) & 1, abort_flag);
+        if (ok) ok = warp_wait(&bars[B_OREADY], 0, abort_flag);
         if (!ok) {
             if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutSoftmax);
         } else {
@@ -732,17 +758,24 @@ cudaError_t launch_bias(int kind, const CUtensorMap& tv, const CUtensorMap& tb, 
                         cudaStream_t st)
 {
     if (kind == BA_BIAS_DENSE) return launch_t<QK, OutT, BA_BIAS_DENSE>(tv, tb, p, smem, st);
+    if (kind == BIAS_RP_FAST) return launch_t<QK, OutT, BIAS_RP_FAST>(tv, tb, p, smem, st);
     if (kind == BA_BIAS_RELPOS2D) return launch_t<QK, OutT, BA_BIAS_RELPOS2D>(tv, tb, p, smem, st);
     return launch_t<QK, OutT, BA_BIAS_NONE>(tv, tb, p, smem, st);
+}
+
+// The kernel variant for an ABI bias kind.
+int kernel_bias(int bias_kind, int gw)
+{
+    return (bias_kind == BA_BIAS_RELPOS2D && gw % BM == 0) ? BIAS_RP_FAST : bias_kind;
 }
 
 }  // namespace
 
 bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d)
 {
-    (void)gh; (void)gw; (void)N;
+    (void)gh; (void)N;
     if (d < 1 || d > 128) return false;
-    return pick_stages(d, bias_kind) >= 2;
+    return pick_stages(d, kernel_bias(bias_kind, gw)) >= 2;
 }
 
 cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
@@ -787,23 +820,22 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     p.out = out;
     p.B = B; p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
     p.n_tiles = ceil_div(N, BN);
-    p.stages = pick_stages(d, bias_kind);
+    const int vb = kernel_bias(bias_kind, gw);
+    p.stages = pick_stages(d, vb);
     p.gh = gh; p.gw = gw;
-    // A 128-row query tile and a 64-key tile then each lie inside one grid row.
-    p.relpos_fast = (bias_kind == BA_BIAS_RELPOS2D && gw % BM == 0) ? 1 : 0;
     p.q_scale = (float)(1.0 / sqrt((double)d));
     p.status = status;
 
     // One CTA per SM: each takes all 512 TMEM columns.
-    size_t smem = smem_bytes(d, bias_kind, p.stages);
+    size_t smem = smem_bytes(d, vb, p.stages);
     if (smem < 120u * 1024u) smem = 120u * 1024u;
 
     const bool f8 = variant != BA_QK_TC_I8;
     if (out_dt == BA_BF16)
-        return f8 ? launch_bias<QK_F8, __nv_bfloat16>(bias_kind, tv, tb, p, smem, st)
-                  : launch_bias<QK_I8, __nv_bfloat16>(bias_kind, tv, tb, p, smem, st);
-    return f8 ? launch_bias<QK_F8, float>(bias_kind, tv, tb, p, smem, st)
-              : launch_bias<QK_I8, float>(bias_kind, tv, tb, p, smem, st);
+        return f8 ? launch_bias<QK_F8, __nv_bfloat16>(vb, tv, tb, p, smem, st)
+                  : launch_bias<QK_I8, __nv_bfloat16>(vb, tv, tb, p, smem, st);
+    return f8 ? launch_bias<QK_F8, float>(vb, tv, tb, p, smem, st)
+              : launch_bias<QK_I8, float>(vb, tv, tb, p, smem, st);
 }
 
 }  // namespace ba
