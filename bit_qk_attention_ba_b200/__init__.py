@@ -15,8 +15,8 @@ import ctypes
 
 from . import _native as N
 
-__all__ = ["pack_qk", "quant_v", "attention_fwd", "scores_debug", "forward", "check_device_status",
-           "words", "vq_ld"]
+__all__ = ["pack_qk", "quant_v", "attention_fwd", "attention_workspace", "workspace_bytes", "scores_debug",
+           "forward", "check_device_status", "words", "vq_ld"]
 
 
 def _torch():
@@ -92,17 +92,43 @@ def _bias_args(bias, bias_kind, ld, grid):
     return bias_kind, _p(bias), int(ld or 0), int(gh), int(gw)
 
 
+def workspace_bytes(B, H, n, d, bias_kind=N.BA_BIAS_NONE, grid=None) -> int:
+    """Device scratch bytes the fused forward needs (ba_attention_workspace_bytes)."""
+    gh, gw = grid if (grid and bias_kind == N.BA_BIAS_RELPOS2D) else (0, 0)
+    nb = N.lib().ba_attention_workspace_bytes(B, H, n, d, int(bias_kind), int(gh), int(gw))
+    if nb < 0:
+        raise ValueError("invalid sizes or bias arguments for the fused forward")
+    return int(nb)
+
+
+def attention_workspace(B, H, n, d, bias_kind=N.BA_BIAS_NONE, grid=None, device=None):
+    """A workspace tensor for attention_fwd (None when none is needed)."""
+    torch = _torch()
+    nb = workspace_bytes(B, H, n, d, bias_kind, grid)
+    if nb == 0:
+        return None
+    # 256-byte alignment: the caching allocator returns 512-byte aligned blocks.
+    return torch.empty((nb,), dtype=torch.uint8, device=device)
+
+
 def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None,
-                  out=None, out_dtype=None, variant=N.BA_QK_AUTO):
-    """Fused forward; returns out [B,H,N,d] (float32 unless out_dtype given)."""
+                  out=None, out_dtype=None, variant=N.BA_QK_AUTO, workspace=None):
+    """Fused forward; returns out [B,H,N,d] (float32 unless out_dtype given).
+    `workspace` (a uint8 CUDA tensor of at least workspace_bytes(...) bytes) is
+    allocated here when not given."""
     torch = _torch()
     _need_cuda(bq, muq, bk, muk, vq, sv)
     B, H, Nn = muq.shape
     if out is None:
         out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=muq.device)
     kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
+    if workspace is None:
+        workspace = attention_workspace(B, H, Nn, d, kind, (gh, gw), device=muq.device)
+    else:
+        _need_cuda(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     N.call("ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
-           B, H, Nn, d, _p(out), _dt(out), int(variant), _stream(muq.device))
+           B, H, Nn, d, _p(workspace), ws_bytes, _p(out), _dt(out), int(variant), _stream(muq.device))
     return out
 
 
@@ -118,14 +144,14 @@ def scores_debug(bq, bk, d, z=None):
 
 
 def forward(q, k, v, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None, out_dtype=None,
-            variant=N.BA_QK_AUTO):
+            variant=N.BA_QK_AUTO, workspace=None):
     """The whole hot path: pack Q, pack K, quantise V, fused attention."""
     d = q.shape[-1]
     bq, muq = pack_qk(q)
     bk, muk = pack_qk(k)
     vq, sv = quant_v(v)
     return attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=bias, bias_kind=bias_kind, ld=ld, grid=grid,
-                         out_dtype=out_dtype or q.dtype, variant=variant)
+                         out_dtype=out_dtype or q.dtype, variant=variant, workspace=workspace)
 
 
 def check_device_status(device=None) -> int:

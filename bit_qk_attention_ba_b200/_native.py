@@ -25,9 +25,11 @@ SIGNATURES = {
     "ba_vq_ld": (_I64, [_I]),
     "ba_pack_qk": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "ba_quant_v": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
-    "ba_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
-    "ba_attention_fwd_variant": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P,
-                                      _I, _I, _P]),
+    "ba_attention_workspace_bytes": (_I64, [_I, _I, _I, _I, _I, _I, _I]),
+    "ba_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I64,
+                              _P, _I, _P]),
+    "ba_attention_fwd_variant": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I64,
+                                      _P, _I, _I, _P]),
     "ba_scores_debug": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "ba_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "ba_status_string": (ctypes.c_char_p, [_I]),

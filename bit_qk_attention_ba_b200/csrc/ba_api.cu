@@ -2,7 +2,8 @@
 //
 // Every entry point validates its arguments on the host before queueing any
 // work, launches asynchronously on the caller's stream and returns a status
-// code; nothing throws across the ABI and nothing is allocated.
+// code; nothing throws across the ABI and nothing is allocated (scratch space
+// is the caller's workspace).
 #include <mutex>
 
 #include "ba_common.cuh"
@@ -23,8 +24,10 @@ cudaError_t launch_attn_simt(const uint32_t* bq, const float* muq, const uint32_
 cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
                            const int8_t* vq, const float* sv, int bias_kind, const float* bias,
                            int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                           void* workspace, int64_t workspace_bytes,
                            void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st);
 bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d);
+int64_t attn_tc_workspace_bytes(int B, int H, int N, int d, int bias_kind, int gh, int gw);
 
 // One status word per device; kernels OR failure bits into it.
 __device__ unsigned g_device_status;
@@ -141,15 +144,25 @@ ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, 
     return from_cuda(launch_scores(bq, bk, B, H, N, d, z, static_cast<cudaStream_t>(stream)));
 }
 
+int64_t ba_attention_workspace_bytes(int B, int H, int N, int d, int bias_kind, int grid_h, int grid_w)
+{
+    if (!sizes_ok(B, H, N, d)) return -1;
+    if (bias_kind != BA_BIAS_NONE && bias_kind != BA_BIAS_DENSE && bias_kind != BA_BIAS_RELPOS2D) return -1;
+    if (bias_kind == BA_BIAS_RELPOS2D && (grid_h < 1 || grid_w < 1 || (int64_t)grid_h * grid_w != N)) return -1;
+    return attn_tc_workspace_bytes(B, H, N, d, bias_kind, grid_h, grid_w);
+}
+
 ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    const uint32_t* bk, const float* muk,
                                    const int8_t* vq, const float* sv,
                                    int bias_kind, const float* bias, int64_t bias_ld,
                                    int grid_h, int grid_w,
                                    int B, int H, int N, int d,
+                                   void* workspace, int64_t workspace_bytes,
                                    void* out, ba_dtype out_dt, int variant, void* stream)
 {
     if (!sizes_ok(B, H, N, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (workspace_bytes < 0 || (workspace_bytes > 0 && !ptr_ok(workspace, 256))) return BA_ERR_INVALID_ARG;
     if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
         !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)))
         return BA_ERR_INVALID_ARG;
@@ -166,11 +179,13 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
         return from_cuda(launch_attn_simt(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
                                           grid_w, B, H, N, d, out, out_dt, st));
     }
+    if (workspace_bytes < attn_tc_workspace_bytes(B, H, N, d, bias_kind, grid_h, grid_w)) return BA_ERR_INVALID_ARG;
     unsigned* status = device_status_ptr();
     if (!status) return BA_ERR_CUDA;
     const cudaError_t e = launch_attn_tc(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
-                                         B, H, N, d, out, out_dt, variant, status, st);
+                                         B, H, N, d, workspace, workspace_bytes, out, out_dt, variant, status, st);
     if (e == cudaErrorNotSupported) return BA_ERR_UNSUPPORTED;
+    if (e == cudaErrorInvalidValue) return BA_ERR_INVALID_ARG;
     return from_cuda(e);
 }
 
@@ -180,10 +195,11 @@ ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
                            int bias_kind, const float* bias, int64_t bias_ld,
                            int grid_h, int grid_w,
                            int B, int H, int N, int d,
+                           void* workspace, int64_t workspace_bytes,
                            void* out, ba_dtype out_dt, void* stream)
 {
     return ba_attention_fwd_variant(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
-                                    B, H, N, d, out, out_dt, BA_QK_AUTO, stream);
+                                    B, H, N, d, workspace, workspace_bytes, out, out_dt, BA_QK_AUTO, stream);
 }
 
 ba_status ba_check_device_status(void* stream, int* code)

@@ -20,28 +20,29 @@
 //     B quantises P~ = exp(S - m_i) against it.  The u8 codes are then the
 //     ones an exact-maximum reference produces, and the int32 PV accumulator
 //     never needs rescaling;
-//   * QK runs on tcgen05.mma from sign bits expanded to +-1 operands in shared
-//     memory (kind::i8 -> s32, or kind::f8f6f4 with e4m3 +-1 -> f32; both are
-//     exact), into double-buffered S tiles in TMEM, so the next tile's QK
-//     overlaps this tile's softmax;
+//   * a staging pre-pass turns the key sign bits into +-1 tensor-core
+//     operands once per call (kind::i8 bytes, or e4m3 +-1 for kind::f8f6f4),
+//     laid out tile by tile in the shared-memory order the QK product reads,
+//     each 64-key tile followed by its key scales; for a 2-D relative-position
+//     bias it also writes every table row reversed, in four copies shifted
+//     by one entry, so any bias window a tile needs is one aligned copy;
+//   * one loader thread moves everything with bulk copies and TMA (key tiles,
+//     bias windows or dense bias boxes, V tiles) into a 2..4-stage ring: the
+//     loader issues no loads or stores of its own;
+//   * QK runs on tcgen05.mma into double-buffered S tiles in TMEM, so the
+//     next tile's QK overlaps this tile's softmax; both kinds are exact;
 //   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (the
-//     softmax writes it over the S tile it came from) and s8 V tiles brought
-//     in by TMA, accumulating in TMEM across all key tiles;
+//     softmax writes it over the S tile it came from) and s8 V tiles,
+//     accumulating in TMEM across all key tiles;
 //   * the softmax pulls each 64-key S tile out of TMEM with one load and does
 //     its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with a 3-input
-//     max;
-//   * the loaders fetch a step's sign bits, scales and bias values into
-//     registers two steps ahead, so global latency overlaps the wait for a
-//     free stage; 2 to 4 stages, as shared memory allows;
-//   * a dense bias tile is staged by TMA with 128-byte swizzle; a 2-D
-//     relative-position bias whose grid width is a multiple of 128 is staged
-//     as reversed, shifted copies of the one table row the tile needs, so each
-//     thread reads its bias as aligned 16-byte vectors.
-// Warps 0-7 run the softmax (two groups of four), warps 8-11 load, warp 12
+//     max; a bias window is read as reversed copies, four keys per 16-byte
+//     load.
+// Warps 0-7 run the softmax (two groups of four), warp 8 loads, warp 9
 // issues the MMAs and owns TMEM.
 //
 // Every wait on an mbarrier is bounded; on a timeout the kernel records a bit
-// in the device status word, tells the other roles to stop, lets issued TMA
+// in the device status word, tells the other roles to stop, lets issued copies
 // and tensor-core work drain, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
@@ -59,37 +60,28 @@ constexpr int BM = 128;                 // query rows per group (= TMEM lanes)
 constexpr int NG = 2;                   // row groups per CTA
 constexpr int BN = 64;                  // keys per tile
 constexpr int MAX_STAGES = 4;
-constexpr int NUM_SOFTMAX_WARPS = 4 * NG;
-constexpr int NUM_LOAD_WARPS = 3;
-constexpr int NUM_LOADERS = 32 * NUM_LOAD_WARPS;
-constexpr int LOAD_WARP0 = NUM_SOFTMAX_WARPS;               // 8
-constexpr int MMA_WARP = LOAD_WARP0 + NUM_LOAD_WARPS;       // 12
-constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 384
-// Warps are given registers in groups of four: 12 warps leave 168 per thread.
+constexpr int NUM_SOFTMAX_WARPS = 4 * NG;                   // 8
+constexpr int LOAD_WARP = NUM_SOFTMAX_WARPS;                // 8
+constexpr int MMA_WARP = LOAD_WARP + 1;                     // 9
+constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 320
+// Warps are given registers in groups of four: 10 warps leave 168 per thread.
 constexpr int MAX_REGS = 168;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int QK_I8 = 0, QK_F8 = 1;
 // Bias variants of the kernel: the three of the ABI, plus a rel-pos fast path
-// for grid widths that are multiples of 128 (tiles then sit inside one grid row).
+// for grid widths that are multiples of 128 (a row group then lies in one grid
+// row and a key tile in one grid row, so its bias is one window of a table row).
 constexpr int BIAS_RP_FAST = 3;
 __host__ __device__ constexpr bool is_relpos(int b) { return b == BA_BIAS_RELPOS2D || b == BIAS_RP_FAST; }
-constexpr int RP_SPAN = BM + BN - 2;    // largest offset inside a rel-pos window (190)
-constexpr int RP_VALS = RP_SPAN + 1;    // values in a window
-constexpr int RP_WIN = 192;             // entries per shifted copy of a window (RP_STRIDE >= RP_WIN)
-constexpr int RP_STRIDE = 200;          // floats between copies (8 words mod 32: conflict-free)
-// Each loader thread builds four consecutive entries of all four copies of
-// one window: it needs seven consecutive window values.
-constexpr int RP_BLOCKS = NG * RP_WIN / 4;                                       // 96
-constexpr int RP_PER_THREAD = 7;
-static_assert(RP_BLOCKS <= NUM_LOADERS, "one rel-pos block per loader thread");
-constexpr int K_PER_THREAD = (2 * BN * 4 + NUM_LOADERS - 1) / NUM_LOADERS;       // sign words, <= 6
-constexpr int MU_PER_THREAD = (2 * BN + NUM_LOADERS - 1) / NUM_LOADERS;          // key scales, <= 2
+constexpr int RP_WIN = 192;             // entries per shifted copy of a window (191 used)
+constexpr int RP_STRIDE = 200;          // floats between copies in shared memory (8 words mod 32)
+constexpr uint32_t RP_COPY_BYTES = RP_WIN * 4;
 
 // Barrier slots.
 enum {
     B_QREADY = 0,
-    B_FULL = 1,                      // [stage] operands, scales, bias (and V in pass B) ready
+    B_FULL = 1,                      // [stage] key tiles, bias (and V in pass B) landed
     B_EMPTY = B_FULL + MAX_STAGES,   // [stage] stage may be overwritten
     B_SFULL = B_EMPTY + MAX_STAGES,  // [NG][2] S tile in TMEM ready
     B_SDONE = B_SFULL + 2 * NG,      // [NG][2] softmax done with the S buffer (pass B: u8 P written into it)
@@ -98,13 +90,20 @@ enum {
     NUM_BARS
 };
 
+// One staged key tile: BN keys x dpad bytes of +-1 operand (K-major core
+// matrices), the BN key scales, and for the general rel-pos bias the BN key
+// offsets rj (2 gw - 1) + cj.
+__host__ __device__ inline uint32_t tile_bytes(int dpad, int bias_kind)
+{
+    return (uint32_t)(BN * dpad + BN * 4 + (bias_kind == BA_BIAS_RELPOS2D ? BN * 4 : 0));
+}
+
 struct Layout {
-    uint32_t stages, kvg;       // pipeline depth; key/value sets per stage (1 or 2)
+    uint32_t stages, kvg, tile; // pipeline depth; key/value sets per stage (1 or 2); staged tile bytes
     uint32_t v, v_bytes;        // [stage][kvg] V tiles (SW64 K-major, dv rows x 64 bytes)
     uint32_t b;                 // [stage][2] dense bias boxes, 16 KB each (SW128)
     uint32_t q, q_bytes;        // [NG] Q operands
-    uint32_t k, k_bytes;        // [stage][kvg] K operands
-    uint32_t muk, koff;         // [stage][kvg][BN], [stage][BN]
+    uint32_t k, k_bytes;        // [stage] kvg staged key tiles
     uint32_t rp;                // [stage][NG][4][RP_STRIDE] rel-pos windows
     uint32_t bars, misc, total;
 };
@@ -116,16 +115,15 @@ __host__ __device__ inline Layout make_layout(int dpad, int dv, int bias_kind, i
     Layout L;
     L.stages = stages;
     L.kvg = (bias_kind == BA_BIAS_DENSE) ? 2u : 1u;
+    L.tile = tile_bytes(dpad, bias_kind == BIAS_RP_FAST ? BA_BIAS_NONE : bias_kind);
     uint32_t off = 0;
     L.v_bytes = align_up((uint32_t)dv * BN, 1024);
     L.v = off; off += stages * L.kvg * L.v_bytes;
     L.b = off; off += (bias_kind == BA_BIAS_DENSE) ? stages * 2 * 16384u : 0u;
     L.q_bytes = align_up((uint32_t)BM * dpad, 1024);
     L.q = off; off += NG * L.q_bytes;
-    L.k_bytes = align_up((uint32_t)BN * dpad, 1024);
-    L.k = off; off += stages * L.kvg * L.k_bytes;
-    L.muk = off; off += stages * L.kvg * BN * 4;
-    L.koff = off; off += (bias_kind == BA_BIAS_RELPOS2D) ? stages * BN * 4 : 0u;
+    L.k_bytes = align_up(L.kvg * L.tile, 128);
+    L.k = off; off += stages * L.k_bytes;
     L.rp = off; off += (bias_kind == BIAS_RP_FAST) ? stages * NG * 4 * RP_STRIDE * 4u : 0u;
     L.bars = off; off += NUM_BARS * 8;
     L.misc = off; off += 16;            // TMEM base address, abort flag
@@ -136,10 +134,10 @@ __host__ __device__ inline Layout make_layout(int dpad, int dv, int bias_kind, i
 struct Params {
     const uint32_t* bq;
     const float* muq;
-    const uint32_t* bk;
-    const float* muk;
+    const uint8_t* kst;      // staged key tiles [B*H][n_tiles][tile]
+    const float* rps;        // staged rel-pos rows [H][2 gh - 1][4][2 gw] (fast path)
     const float* sv;
-    const float* table;      // 2-D relative-position table (global)
+    const float* table;      // 2-D relative-position table (general rel-pos path)
     void* out;
     int B, H, N, d, W, dpad, dv, n_tiles, stages;
     int gh, gw;
@@ -302,15 +300,6 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
     }
 }
 
-// What one loader thread fetches from global memory for one step, held in
-// registers until the stage is free.
-struct Prefetch {
-    uint32_t kbits[K_PER_THREAD];   // sign words of this thread's (key, word) items
-    float muk[MU_PER_THREAD];       // key scales
-    int koff[MU_PER_THREAD];        // keys' rel-pos offsets (general rel-pos path)
-    float rp[RP_PER_THREAD];        // seven consecutive reversed-window values
-};
-
 template <int QK, typename OutT, int BIAS>
 __global__ void __maxnreg__(MAX_REGS)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
@@ -331,13 +320,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     const int S = p.stages;
     const int chunks = p.dpad / 16;
     const int h = PAIR ? (int)blockIdx.y : (int)(blockIdx.y % p.H);
-    const float* tab_h = is_relpos(BIAS)
+    const float* tab_h = (BIAS == BA_BIAS_RELPOS2D)
                              ? p.table + (size_t)h * (2 * p.gh - 1) * (2 * p.gw - 1) : nullptr;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_QREADY], NUM_SOFTMAX_WARPS);
         for (int s = 0; s < S; ++s) {
-            mbar_init(&bars[B_FULL + s], NUM_LOAD_WARPS);
+            mbar_init(&bars[B_FULL + s], 1);
             mbar_init(&bars[B_EMPTY + s], NUM_SOFTMAX_WARPS + 1);
         }
         for (int b = 0; b < 2 * NG; ++b) {
@@ -353,7 +342,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == LOAD_WARP0 && lane == 0) {
+    if (warp == LOAD_WARP && lane == 0) {
         prefetch_tmap(&tm_v);
         if (BIAS == BA_BIAS_DENSE) prefetch_tmap(&tm_b);
     }
@@ -362,159 +351,76 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
-        // ---------------------------------------------------------------- loaders
-        // Every loader thread owns fixed items of each stage: up to four (key
-        // set, key, word) sign words, one key scale, and up to three values of
-        // the rel-pos windows.  Their addresses are worked out once here; per
-        // step only the key offset j0 moves.  Global loads for step u + 2 are
-        // issued right after step u is stored, so their latency overlaps the
-        // wait for a free stage.
-        const int lw = warp - LOAD_WARP0;
-        const int ltid = lw * 32 + lane;
-        int kvbh0, kvbh1;
-        {
-            int q0x;
-            bool ex;
-            group_coords<PAIR>(p, 0, kvbh0, q0x, ex);
-            kvbh1 = kvbh0;
-            if (KVG > 1) group_coords<PAIR>(p, 1, kvbh1, q0x, ex);
-        }
-        const int kitems = KVG * BN * W;
-        const uint32_t* kbase[K_PER_THREAD];
-        int krow[K_PER_THREAD];
-        uint32_t kdst[K_PER_THREAD];
+    if (warp == LOAD_WARP) {
+        // ---------------------------------------------------------------- loader
+        // One thread fills stage u % S for step u: the staged key tile(s), the
+        // bias of the tile (two windows of reversed table rows, one per group,
+        // each in four shifted copies; or two dense-bias boxes), and in pass B
+        // the V tile(s).  All copies complete on the stage's FULL barrier.
+        if (lane == 0) {
+            int kvbh0, kvbh1, q0g[NG];
+            {
+                bool ex;
+                group_coords<PAIR>(p, 0, kvbh0, q0g[0], ex);
+                group_coords<PAIR>(p, 1, kvbh1, q0g[1], ex);
+                if (!PAIR) kvbh1 = kvbh0;
+            }
+            const size_t row_len = 2 * (size_t)p.gw;
+            const float* rps_h = (BIAS == BIAS_RP_FAST) ? p.rps + (size_t)h * (2 * p.gh - 1) * 4 * row_len : nullptr;
+            int rp_ri[NG], rp_ci[NG];
 #pragma unroll
-        for (int k = 0; k < K_PER_THREAD; ++k) {
-            const int e = ltid + k * NUM_LOADERS;
-            const int x = e / (BN * W), rem = e - x * (BN * W);
-            const int r = rem / W, w = rem - r * W;
-            krow[k] = (e < kitems) ? r : (1 << 30);          // never valid
-            kbase[k] = p.bk + ((size_t)(x ? kvbh1 : kvbh0) * N + r) * W + w;
-            kdst[k] = (uint32_t)(x * L.k_bytes) + core_off(r, 2 * w, chunks);
-        }
-        int mu_row[MU_PER_THREAD];
-        const float* mu_base[MU_PER_THREAD];
-#pragma unroll
-        for (int k = 0; k < MU_PER_THREAD; ++k) {
-            const int e = ltid + k * NUM_LOADERS;
-            mu_row[k] = (e < KVG * BN) ? e % BN : (1 << 30);   // never valid
-            mu_base[k] = p.muk + (size_t)((e / BN) ? kvbh1 : kvbh0) * N + e % BN;
-        }
-        // Rel-pos window block of this thread: group rp_g, entries rp_y..rp_y+3
-        // of each copy, built from Rr[rp_y .. rp_y + 6] (Rr = reversed window).
-        const float* rp_src = tab_h;
-        int rp_y = -1, rp_g = 0;
-        if (BIAS == BIAS_RP_FAST && ltid < RP_BLOCKS) {
-            rp_g = ltid / (RP_WIN / 4);
-            rp_y = (ltid - rp_g * (RP_WIN / 4)) * 4;
-            int bhg, q0g;
-            bool ex;
-            group_coords<PAIR>(p, rp_g, bhg, q0g, ex);
-            if (q0g >= N) q0g = N - BM;              // an empty group still reads inside the table
-            const int ri = q0g / p.gw, ci0 = q0g - ri * p.gw;
-            // Rr[v] = R[xlo + RP_SPAN - v] with R the table row of offset ri - rj
-            // and xlo = ci0 - cj0 - (BN - 1) + gw - 1; only the key-tile part
-            // rj * (2 gw - 1) + cj0 changes per step.
-            rp_src = tab_h + (ptrdiff_t)(ri + p.gh - 1) * (2 * p.gw - 1) + ci0 - (BN - 1) + p.gw - 1 + RP_SPAN - rp_y;
-        }
-
-        auto fetch = [&](int u, Prefetch& f) {
-            const int t = (u >= T) ? u - T : u;
-            const int j0 = t * BN;
-#pragma unroll
-            for (int k = 0; k < K_PER_THREAD; ++k)
-                f.kbits[k] = (j0 + krow[k] < N) ? __ldg(kbase[k] + (size_t)j0 * W) : 0u;
-#pragma unroll
-            for (int k = 0; k < MU_PER_THREAD; ++k) {
-                f.muk[k] = (j0 + mu_row[k] < N) ? __ldg(mu_base[k] + j0) : 0.f;
-                f.koff[k] = 0;
-                const int e = ltid + k * NUM_LOADERS;
-                if (BIAS == BA_BIAS_RELPOS2D && e < BN) {
-                    const int jj = min(j0 + e, N - 1);
-                    const int rj = jj / p.gw, cj = jj - rj * p.gw;
-                    f.koff[k] = rj * (2 * p.gw - 1) + cj;
+            for (int g = 0; g < NG; ++g) {
+                const int q0 = (q0g[g] < N) ? q0g[g] : N - BM;     // an empty group still reads inside the table
+                rp_ri[g] = (BIAS == BIAS_RP_FAST) ? q0 / p.gw : 0;
+                rp_ci[g] = (BIAS == BIAS_RP_FAST) ? q0 - rp_ri[g] * p.gw : 0;
+            }
+            const uint32_t step_bytes = KVG * L.tile + (BIAS == BIAS_RP_FAST ? NG * 4 * RP_COPY_BYTES : 0u) +
+                                        (BIAS == BA_BIAS_DENSE ? 2 * 16384u : 0u);
+            const uint32_t v_bytes = (uint32_t)(KVG * p.dv * BN);
+            int issued = 0;
+            for (int u = 0; u < U; ++u) {
+                const int s = u % S;
+                const bool pass_b = u >= T;
+                const int t = pass_b ? u - T : u;
+                const int j0 = t * BN;
+                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], (u / S - 1) & 1, abort_flag)) {
+                    fail(abort_flag, p.status, kStatusTimeoutProducer);
+                    break;
                 }
-            }
-            if (BIAS == BIAS_RP_FAST) {
-                const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
-                const ptrdiff_t shift = (ptrdiff_t)rj * (2 * p.gw - 1) + cj0;
+                uint64_t* full = &bars[B_FULL + s];
+                mbar_arrive_expect_tx(full, step_bytes + (pass_b ? v_bytes : 0u));
+                uint8_t* kdst = smem + L.k + s * L.k_bytes;
+                bulk_load(kdst, p.kst + ((size_t)kvbh0 * T + t) * L.tile, L.tile, full);
+                if (KVG > 1) bulk_load(kdst + L.tile, p.kst + ((size_t)kvbh1 * T + t) * L.tile, L.tile, full);
+                if (BIAS == BIAS_RP_FAST) {
+                    // Window of group g: entries xs .. xs + 191 of the reversed
+                    // row for ri - rj, xs = gw - 128 - (ci0 - cj0), in each copy.
+                    const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
 #pragma unroll
-                for (int k = 0; k < RP_PER_THREAD; ++k)
-                    f.rp[k] = (rp_y >= 0 && rp_y + k <= RP_SPAN) ? __ldg(rp_src - shift - k) : 0.f;
-            }
-        };
-
-        auto step = [&](int u, const Prefetch& f) -> bool {
-            const int s = u % S, use = u / S;
-            const bool pass_b = u >= T;
-            const int t = pass_b ? u - T : u;
-            const int j0 = t * BN;
-            if (u >= S && !warp_wait(&bars[B_EMPTY + s], (use - 1) & 1, abort_flag)) {
-                if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutProducer);
-                return false;
-            }
-            if (lw == 0 && lane == 0) {
-                const uint32_t bytes = (pass_b ? (uint32_t)(KVG * p.dv * BN) : 0u) +
-                                       (BIAS == BA_BIAS_DENSE ? 2 * 16384u : 0u);
-                if (bytes) mbar_expect_tx(&bars[B_FULL + s], bytes);
-                if (pass_b) {
-                    tma_load_3d(smem + L.v + (s * KVG) * L.v_bytes, &tm_v, &bars[B_FULL + s], j0, 0, kvbh0);
-                    if (KVG > 1)
-                        tma_load_3d(smem + L.v + (s * KVG + 1) * L.v_bytes, &tm_v, &bars[B_FULL + s], j0, 0, kvbh1);
+                    for (int g = 0; g < NG; ++g) {
+                        const int rho = rp_ri[g] - rj + p.gh - 1;
+                        const int xs = p.gw - BM - (rp_ci[g] - cj0);
+                        const float* src = rps_h + (size_t)rho * 4 * row_len + xs;
+                        float* dst = reinterpret_cast<float*>(smem + L.rp) + (size_t)(s * NG + g) * 4 * RP_STRIDE;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            bulk_load(dst + m * RP_STRIDE, src + m * row_len, RP_COPY_BYTES, full);
+                    }
                 }
                 if (BIAS == BA_BIAS_DENSE)
                     for (int bx = 0; bx < 2; ++bx)
-                        tma_load_3d(smem + L.b + (s * 2 + bx) * 16384, &tm_b, &bars[B_FULL + s],
-                                    j0 + 32 * bx, (int)blockIdx.x * BM, h);
-            }
-            uint8_t* kop = smem + L.k + s * KVG * L.k_bytes;
-#pragma unroll
-            for (int k = 0; k < K_PER_THREAD; ++k) {
-                if (krow[k] < BN) {
-                    *reinterpret_cast<uint4*>(kop + kdst[k]) = expand16<QK>(f.kbits[k] & 0xFFFFu, 0xFFFFu);
-                    *reinterpret_cast<uint4*>(kop + kdst[k] + 128) = expand16<QK>(f.kbits[k] >> 16, 0xFFFFu);
+                        tma_load_3d(smem + L.b + (s * 2 + bx) * 16384, &tm_b, full, j0 + 32 * bx,
+                                    (int)blockIdx.x * BM, h);
+                if (pass_b) {
+                    tma_load_3d(smem + L.v + (s * KVG) * L.v_bytes, &tm_v, full, j0, 0, kvbh0);
+                    if (KVG > 1) tma_load_3d(smem + L.v + (s * KVG + 1) * L.v_bytes, &tm_v, full, j0, 0, kvbh1);
                 }
+                issued = u + 1;
             }
-#pragma unroll
-            for (int k = 0; k < MU_PER_THREAD; ++k) {
-                const int e = ltid + k * NUM_LOADERS;
-                if (e < KVG * BN) {
-                    reinterpret_cast<float*>(smem + L.muk)[s * KVG * BN + e] = f.muk[k];
-                    if (BIAS == BA_BIAS_RELPOS2D && e < BN)
-                        reinterpret_cast<int*>(smem + L.koff)[s * BN + e] = f.koff[k];
-                }
-            }
-            if (BIAS == BIAS_RP_FAST) {
-                // Copy m of group g holds Rr[y + m] at entry y.
-                if (rp_y >= 0) {
-                    float* dst = reinterpret_cast<float*>(smem + L.rp) + ((size_t)s * NG * 4 + rp_g * 4) * RP_STRIDE + rp_y;
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<float4*>(dst + m * RP_STRIDE) =
-                            make_float4(f.rp[m], f.rp[m + 1], f.rp[m + 2], f.rp[m + 3]);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
-            return true;
-        };
-
-        Prefetch pa, pb;
-        fetch(0, pa);
-        if (U > 1) fetch(1, pb);
-        for (int u = 0; u < U; u += 2) {
-            if (!step(u, pa)) break;
-            if (u + 2 < U) fetch(u + 2, pa);
-            if (u + 1 >= U) break;
-            if (!step(u + 1, pb)) break;
-            if (u + 3 < U) fetch(u + 3, pb);
-        }
-        // On an abort, let TMA copies already issued land before the CTA exits.
-        if (*abort_flag && lw == 0 && lane == 0) {
-            for (int u = (U > S ? U - S : 0); u < U; ++u)
-                mbar_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
+            // On an abort, let copies already issued land before the CTA exits.
+            if (*abort_flag)
+                for (int u = (issued > S ? issued - S : 0); u < issued; ++u)
+                    mbar_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
@@ -530,7 +436,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
             const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
             const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
-            const uint32_t q_step = L.q_bytes >> 4, k_step = L.k_bytes >> 4, v_step = L.v_bytes >> 4;
+            const uint32_t q_step = L.q_bytes >> 4, v_step = L.v_bytes >> 4;
             const int kq = p.dpad / 32;
             auto issue_qk = [&](int u) -> bool {
                 const int s = u % S, buf = u & 1;
@@ -541,7 +447,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 tc_fence_after();
                 for (int g = 0; g < NG; ++g) {
                     const uint64_t dq = dq0 + g * q_step;
-                    const uint64_t dk = dk0 + (s * KVG + (PAIR ? g : 0)) * k_step;
+                    const uint64_t dk = dk0 + ((s * L.k_bytes + (PAIR ? g : 0) * L.tile) >> 4);
                     const uint32_t d_tmem = tmem + (2 * g + buf) * BN;
                     for (int kk = 0; kk < kq; ++kk)
                         mma_ss<QK>(d_tmem, dq + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
@@ -633,8 +539,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             if (!ok) break;
             tc_fence_after();
             const bool ragged = j0 + BN > N;
-            const float* muk_s = reinterpret_cast<const float*>(smem + L.muk) + (s * KVG + kvx) * BN;
-            const int* koff_s = reinterpret_cast<const int*>(smem + L.koff) + s * BN;
+            const uint8_t* tile_s = smem + L.k + s * L.k_bytes + kvx * L.tile;
+            const float* muk_s = reinterpret_cast<const float*>(tile_s + BN * p.dpad);
+            const int* koff_s = reinterpret_cast<const int*>(tile_s + BN * p.dpad + BN * 4);
             const uint8_t* bsm_row = smem + L.b + s * 2 * 16384 + r * 128;
             const float* rpc = (BIAS == BIAS_RP_FAST)
                 ? reinterpret_cast<const float*>(smem + L.rp) + (size_t)s * NG * 4 * RP_STRIDE + rp_off : nullptr;
@@ -769,6 +676,74 @@ int kernel_bias(int bias_kind, int gw)
     return (bias_kind == BA_BIAS_RELPOS2D && gw % BM == 0) ? BIAS_RP_FAST : bias_kind;
 }
 
+// Workspace layout: staged key tiles, then (fast rel-pos path) staged table rows.
+struct Workspace {
+    int64_t kst_bytes, rps_off, rps_bytes, total;
+};
+
+Workspace workspace_layout(int B, int H, int N, int d, int bias_kind, int gh, int gw)
+{
+    const int vb = kernel_bias(bias_kind, gw);
+    Workspace w;
+    const int64_t tile = tile_bytes(32 * words_for(d), vb == BIAS_RP_FAST ? BA_BIAS_NONE : vb);
+    w.kst_bytes = (int64_t)B * H * ceil_div(N, BN) * tile;
+    w.rps_off = round_up64(w.kst_bytes, 256);
+    w.rps_bytes = (vb == BIAS_RP_FAST) ? (int64_t)H * (2 * gh - 1) * 4 * (2 * (int64_t)gw) * 4 : 0;
+    w.total = w.rps_off + w.rps_bytes;
+    return w;
+}
+
+// Staging of the key side, one CTA per (64-key tile, batch*head): +-1 operand
+// bytes in core-matrix order, the key scales (0 past N), and for the general
+// rel-pos bias the key offsets rj (2 gw - 1) + cj.  Keys past N get operand
+// rows of their (zero) sign bits; the kernel masks them out of the softmax.
+template <int QK>
+__global__ void __launch_bounds__(128)
+stage_k_kernel(const uint32_t* __restrict__ bk, const float* __restrict__ muk, int N, int W, int T,
+               int koff_gw, uint32_t tile, uint8_t* __restrict__ kst)
+{
+    const int t = blockIdx.x;
+    const size_t bh = blockIdx.y;
+    uint8_t* dst = kst + (bh * T + t) * tile;
+    const int dpad = 32 * W, chunks = 2 * W;
+    for (int e = threadIdx.x; e < BN * W; e += blockDim.x) {
+        const int r = e / W, w = e - r * W;
+        const int j = t * BN + r;
+        const uint32_t bits = (j < N) ? __ldg(bk + (bh * N + j) * W + w) : 0u;
+        *reinterpret_cast<uint4*>(dst + core_off(r, 2 * w, chunks)) = expand16<QK>(bits & 0xFFFFu, 0xFFFFu);
+        *reinterpret_cast<uint4*>(dst + core_off(r, 2 * w + 1, chunks)) = expand16<QK>(bits >> 16, 0xFFFFu);
+    }
+    float* mu = reinterpret_cast<float*>(dst + BN * dpad);
+    int* ko = reinterpret_cast<int*>(dst + BN * dpad + BN * 4);
+    for (int r = threadIdx.x; r < BN; r += blockDim.x) {
+        const int j = t * BN + r;
+        mu[r] = (j < N) ? __ldg(muk + bh * N + j) : 0.f;
+        if (koff_gw > 0) {
+            const int jj = (j < N) ? j : N - 1;
+            const int rj = jj / koff_gw;
+            ko[r] = rj * (2 * koff_gw - 1) + (jj - rj * koff_gw);
+        }
+    }
+}
+
+// Staging of the rel-pos table for the fast path: for head h and row rho of
+// the table, copy m holds the reversed row shifted by m,
+// rps[h][rho][m][x] = table[h][rho][2 gw - 2 - (x + m)] (0 past the row's end).
+__global__ void __launch_bounds__(256)
+stage_rp_kernel(const float* __restrict__ table, int gh, int gw, int64_t total, float* __restrict__ rps)
+{
+    const int64_t row_len = 2 * (int64_t)gw;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t x = i % row_len;
+        const int64_t rest = i / row_len;              // (h (2 gh - 1) + rho) * 4 + m
+        const int m = (int)(rest & 3);
+        const int64_t row = rest >> 2;                 // h (2 gh - 1) + rho
+        const int64_t src = x + m;
+        rps[i] = (src <= 2 * (int64_t)gw - 2) ? __ldg(table + row * (2 * gw - 1) + (2 * gw - 2 - src)) : 0.f;
+    }
+}
+
 }  // namespace
 
 bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d)
@@ -778,17 +753,28 @@ bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d)
     return pick_stages(d, kernel_bias(bias_kind, gw)) >= 2;
 }
 
+int64_t attn_tc_workspace_bytes(int B, int H, int N, int d, int bias_kind, int gh, int gw)
+{
+    if (!attn_tc_supports(bias_kind, gh, gw, N, d)) return 0;
+    return workspace_layout(B, H, N, d, bias_kind, gh, gw).total;
+}
+
 cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
                            const int8_t* vq, const float* sv, int bias_kind, const float* bias,
                            int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                           void* workspace, int64_t workspace_bytes,
                            void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st)
 {
     if (!attn_tc_supports(bias_kind, gh, gw, N, d)) return cudaErrorNotSupported;
+    const Workspace ws = workspace_layout(B, H, N, d, bias_kind, gh, gw);
+    if (workspace == nullptr || workspace_bytes < ws.total) return cudaErrorInvalidValue;
     auto encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
     const int BH = B * H;
     const int dv = dv_of(d);
     const int64_t ldv = round_up64(N, 16);
+    const int vb = kernel_bias(bias_kind, gw);
+    const bool f8 = variant != BA_QK_TC_I8;
 
     CUtensorMap tv, tb;
     memset(&tv, 0, sizeof(tv));
@@ -815,22 +801,43 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     }
 
     Params p;
-    p.bq = bq; p.muq = muq; p.bk = bk; p.muk = muk; p.sv = sv;
+    p.bq = bq; p.muq = muq; p.sv = sv;
+    p.kst = static_cast<const uint8_t*>(workspace);
+    p.rps = (vb == BIAS_RP_FAST) ? reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + ws.rps_off)
+                                 : nullptr;
     p.table = bias_kind == BA_BIAS_RELPOS2D ? bias : nullptr;
     p.out = out;
     p.B = B; p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
     p.n_tiles = ceil_div(N, BN);
-    const int vb = kernel_bias(bias_kind, gw);
     p.stages = pick_stages(d, vb);
     p.gh = gh; p.gw = gw;
     p.q_scale = (float)(1.0 / sqrt((double)d));
     p.status = status;
 
+    // Staging pre-passes (same stream, so the attention kernel sees them).
+    {
+        const uint32_t tile = tile_bytes(p.dpad, vb == BIAS_RP_FAST ? BA_BIAS_NONE : vb);
+        uint8_t* kst = static_cast<uint8_t*>(workspace);
+        const int koff_gw = (vb == BA_BIAS_RELPOS2D) ? gw : 0;
+        dim3 grid(p.n_tiles, BH);
+        if (f8) stage_k_kernel<QK_F8><<<grid, 128, 0, st>>>(bk, muk, N, p.W, p.n_tiles, koff_gw, tile, kst);
+        else stage_k_kernel<QK_I8><<<grid, 128, 0, st>>>(bk, muk, N, p.W, p.n_tiles, koff_gw, tile, kst);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        if (vb == BIAS_RP_FAST) {
+            const int64_t total = ws.rps_bytes / 4;
+            const int blocks = (int)((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
+            stage_rp_kernel<<<blocks, 256, 0, st>>>(bias, gh, gw, total,
+                                                     reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.rps_off));
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+    }
+
     // One CTA per SM: each takes all 512 TMEM columns.
     size_t smem = smem_bytes(d, vb, p.stages);
     if (smem < 120u * 1024u) smem = 120u * 1024u;
 
-    const bool f8 = variant != BA_QK_TC_I8;
     if (out_dt == BA_BF16)
         return f8 ? launch_bias<QK_F8, __nv_bfloat16>(vb, tv, tb, p, smem, st)
                   : launch_bias<QK_I8, __nv_bfloat16>(vb, tv, tb, p, smem, st);

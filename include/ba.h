@@ -15,7 +15,8 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
  *     in the layout stated and aligned to their element size; the int8 V codes
  *     and a dense bias must be 16-byte aligned (they are read by the tensor
- *     memory accelerator).  The library allocates no device memory and never
+ *     memory accelerator).  The library allocates no device memory (the fused
+ *     forward's scratch space is a caller workspace, see below) and never
  *     synchronises: work is queued on `stream` (a cudaStream_t passed as
  *     void*; NULL is the legacy default stream).
  *   - Arguments are validated before anything is queued; an invalid call
@@ -95,6 +96,16 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
                      int8_t* vq, float* sv, void* stream);
 
 /*
+ * Bytes of device workspace the fused forward needs for this problem (0 when
+ * the shape runs on the CUDA-core path, which needs none); -1 for invalid
+ * sizes or bias arguments.  The workspace holds the key side staged for the
+ * tensor cores: +-1 operand tiles with their key scales, and for a 2-D
+ * relative-position bias with grid_w a multiple of 128 the table rows
+ * reversed in four shifted copies.  It is rewritten by every call.
+ */
+int64_t ba_attention_workspace_bytes(int B, int H, int N, int d, int bias_kind, int grid_h, int grid_w);
+
+/*
  * KD1-KD3 + FW -- the fused forward.  For every (b, h, i):
  *   z_ij  = s_i . t_j = d - 2 popcount(bq_i XOR bk_j)                   (KD1)
  *   S_ij  = muq_i muk_j z_ij / sqrt(d) + b_ij                            (KD2)
@@ -108,6 +119,10 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
  *   4).  RELPOS2D: token i sits at (i / grid_w, i % grid_w), N must equal
  *   grid_h * grid_w, and b_ij = table[h][(ri - rj + grid_h - 1) *
  *   (2 grid_w - 1) + (ci - cj + grid_w - 1)].
+ * workspace: device scratch of at least ba_attention_workspace_bytes(...)
+ *   bytes, 256-byte aligned (may be NULL when that size is 0); owned by the
+ *   caller, used only by work queued on `stream` by this call.  Too small a
+ *   workspace returns BA_ERR_INVALID_ARG.
  * out: [B, H, N, d] in out_dt (BA_F32 or BA_BF16).
  * The keys are swept twice inside the kernel (maximum first, then P and PV),
  * so pq is quantised against the exact maximum rather than a running one;
@@ -119,6 +134,7 @@ ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
                            int bias_kind, const float* bias, int64_t bias_ld,
                            int grid_h, int grid_w,
                            int B, int H, int N, int d,
+                           void* workspace, int64_t workspace_bytes,
                            void* out, ba_dtype out_dt, void* stream);
 
 /* Same computation with an explicit QK contraction path (ba_qk_variant);
@@ -129,6 +145,7 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    int bias_kind, const float* bias, int64_t bias_ld,
                                    int grid_h, int grid_w,
                                    int B, int H, int N, int d,
+                                   void* workspace, int64_t workspace_bytes,
                                    void* out, ba_dtype out_dt, int variant, void* stream);
 
 /*

@@ -59,7 +59,7 @@ def test_bad_sizes_rejected(lib, B, H, N, d):
     assert lib.ba_quant_v(FAKE, 1, B, H, N, d, FAKE, FAKE, None) == 1
     assert lib.ba_scores_debug(FAKE, FAKE, B, H, N, d, FAKE, None) == 1
     assert lib.ba_attention_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, 0, 0, 0,
-                                B, H, N, d, FAKE, 0, None) == 1
+                                B, H, N, d, None, 0, FAKE, 0, None) == 1
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
@@ -68,23 +68,51 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.ba_quant_v(FAKE, 1, 1, 1, 8, 64, MIS, FAKE, None) == 1
     assert lib.ba_scores_debug(FAKE, None, 1, 1, 8, 64, FAKE, None) == 1
     args = [FAKE] * 6
-    assert lib.ba_attention_fwd(*args[:5], None, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
-    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, MIS, 0, None) == 1
+    assert lib.ba_attention_fwd(*args[:5], None, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, MIS, 0, None) == 1
 
 
 def test_bad_dtypes_and_bias_rejected(lib):
     assert lib.ba_pack_qk(FAKE, 7, 1, 1, 8, 64, FAKE, FAKE, None) == 1
     args = [FAKE] * 6
     # dense bias: ld < N, ld not a multiple of 4, null table
-    assert lib.ba_attention_fwd(*args, 1, FAKE, 4, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
-    assert lib.ba_attention_fwd(*args, 1, FAKE, 9, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
-    assert lib.ba_attention_fwd(*args, 1, None, 8, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 1, FAKE, 4, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 1, FAKE, 9, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 1, None, 8, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     # rel-pos: N must equal grid_h * grid_w
-    assert lib.ba_attention_fwd(*args, 2, FAKE, 0, 3, 3, 1, 1, 8, 64, FAKE, 0, None) == 1
-    assert lib.ba_attention_fwd(*args, 5, FAKE, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 2, FAKE, 0, 3, 3, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 5, FAKE, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     # out dtype and unknown QK variant
-    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 9, None) == 1
-    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, FAKE, 0, 2, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 9, None) == 1
+    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, 2, None) == 1
+
+
+def test_workspace_size_query(lib):
+    """Size of the staged key side: 64-key tiles of +-1 operand bytes plus key
+    scales (plus key offsets for the general rel-pos bias), and for a rel-pos
+    grid width that is a multiple of 128 four shifted copies of every
+    reversed table row."""
+    ws = lib.ba_attention_workspace_bytes
+    tiles = 16384 // 64
+    kst = 4 * 12 * tiles * (64 * 64 + 64 * 4)
+    rps = 12 * (2 * 128 - 1) * 4 * (2 * 128) * 4
+    assert ws(4, 12, 16384, 64, 2, 128, 128) == kst + rps
+    assert ws(4, 12, 16384, 64, 0, 0, 0) == kst
+    assert ws(32, 12, 577, 64, 1, 0, 0) == 32 * 12 * 10 * (64 * 64 + 256)
+    assert ws(2, 2, 300, 72, 2, 15, 20) == 2 * 2 * 5 * (64 * 96 + 256 + 256)   # general rel-pos: offsets too
+    assert ws(0, 1, 8, 64, 0, 0, 0) == -1
+    assert ws(1, 1, 8, 64, 2, 3, 3) == -1
+    assert ws(1, 1, 8, 64, 7, 0, 0) == -1
+
+
+def test_workspace_checked_before_launch(lib):
+    args = [FAKE] * 6
+    need = lib.ba_attention_workspace_bytes(1, 1, 256, 64, 0, 0, 0)
+    assert need > 0
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 256, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 256, 64, FAKE, need - 16, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 256, 64, MIS, need, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 256, 64, FAKE, -1, FAKE, 0, None) == 1
 
 
 def test_product_path_has_no_oracle_or_fallback():
