@@ -15,8 +15,8 @@ import ctypes
 
 from . import _native as N
 
-__all__ = ["pack_qk", "quant_v", "attention_fwd", "attention_workspace", "workspace_bytes", "scores_debug",
-           "forward", "check_device_status", "words", "vq_ld"]
+__all__ = ["pack_qk", "quant_v", "attention_fwd", "attention_fwd_noalloc", "attention_workspace",
+           "workspace_bytes", "scores_debug", "forward", "check_device_status", "words", "vq_ld"]
 
 
 def _torch():
@@ -129,6 +129,21 @@ def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NO
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     N.call("ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
            B, H, Nn, d, _p(workspace), ws_bytes, _p(out), _dt(out), int(variant), _stream(muq.device))
+    return out
+
+
+def attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None,
+                          out=None, out_dtype=None):
+    """attention_fwd with the library's own static scratch instead of a
+    workspace (ba_attention_fwd_noalloc)."""
+    torch = _torch()
+    _need_cuda(bq, muq, bk, muk, vq, sv)
+    B, H, Nn = muq.shape
+    if out is None:
+        out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=muq.device)
+    kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
+    N.call("ba_attention_fwd_noalloc", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
+           B, H, Nn, d, _p(out), _dt(out), _stream(muq.device))
     return out
 
 

@@ -30,6 +30,8 @@ SIGNATURES = {
                               _P, _I, _P]),
     "ba_attention_fwd_variant": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I64,
                                       _P, _I, _I, _P]),
+    "ba_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I,
+                                      _P]),
     "ba_scores_debug": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "ba_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "ba_status_string": (ctypes.c_char_p, [_I]),

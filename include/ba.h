@@ -149,6 +149,22 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    void* out, ba_dtype out_dt, int variant, void* stream);
 
 /*
+ * ba_attention_fwd without a caller workspace: the staging goes to scratch
+ * space the library owns, a static device array of 80 MiB (83886080 bytes)
+ * per device, reserved when this entry point is first used.  Returns
+ * BA_ERR_UNSUPPORTED when ba_attention_workspace_bytes(...) exceeds that.
+ * Calls share the array: at most one may be in flight per device at a time
+ * (queue them on one stream, or synchronise between them).
+ */
+ba_status ba_attention_fwd_noalloc(const uint32_t* bq, const float* muq,
+                                   const uint32_t* bk, const float* muk,
+                                   const int8_t* vq, const float* sv,
+                                   int bias_kind, const float* bias, int64_t bias_ld,
+                                   int grid_h, int grid_w,
+                                   int B, int H, int N, int d,
+                                   void* out, ba_dtype out_dt, void* stream);
+
+/*
  * KD1 -- the integer binary score matrix, for checking and debugging.
  *   z : [B, H, N, N] int32, z[b][h][i][j] = d - 2 popcount(bq_i XOR bk_j).
  */

@@ -1,0 +1,77 @@
+"""ba_attention_fwd_noalloc: the fused forward on the library's static scratch.
+
+Collected last on purpose: the first call reserves the library's static
+scratch array on the device, so the other GPU tests run before it.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle as O
+from bit_qk_attention_ba_b200 import _native as NAT
+from bit_qk_attention_ba_b200.workloads import BIAS_KIND, Workload, make_inputs
+
+STATIC_BYTES = 80 << 20
+FAKE = ctypes.c_void_p(1 << 20)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    try:
+        return NAT.load()
+    except ImportError as e:
+        pytest.skip(str(e))
+
+
+def test_noalloc_rejects_before_any_launch(lib):
+    args = [FAKE] * 6
+    # bad sizes
+    assert lib.ba_attention_fwd_noalloc(*args, 0, None, 0, 0, 0, 0, 1, 8, 64, FAKE, 0, None) == NAT.BA_ERR_INVALID_ARG
+    # a problem whose staged key side exceeds the static array: 8 x 16 heads of 16384 keys
+    need = lib.ba_attention_workspace_bytes(8, 16, 16384, 64, 0, 0, 0)
+    assert need > STATIC_BYTES
+    assert lib.ba_attention_fwd_noalloc(*args, 0, None, 0, 0, 0, 8, 16, 16384, 64, FAKE, 0,
+                                        None) == NAT.BA_ERR_UNSUPPORTED
+    # the largest benchmark workload fits
+    assert lib.ba_attention_workspace_bytes(4, 12, 16384, 64, 2, 128, 128) <= STATIC_BYTES
+
+
+CASES = [
+    Workload("na_dense", 2, 2, 300, 64, bias="dense", bias_std=0.3),
+    Workload("na_relpos_fast", 1, 2, 256, 64, bias="relpos2d", grid=(2, 128), bias_std=0.3),
+    Workload("na_none_d72", 1, 3, 200, 72, bias="none"),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_noalloc_matches_workspace_path_and_oracle(w):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import bit_qk_attention_ba_b200 as ba
+    dev = torch.device("cuda:0")
+    inp = make_inputs(w)
+    g = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev).to(torch.bfloat16)
+    q, k, v = g(inp["q"]), g(inp["k"]), g(inp["v"])
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
+    kind = BIAS_KIND[w.bias]
+    bq, muq = ba.pack_qk(q)
+    bk, muk = ba.pack_qk(k)
+    vq, sv = ba.quant_v(v)
+    ref = ba.attention_fwd(bq, muq, bk, muk, vq, sv, w.d, bias=bias, bias_kind=kind, ld=inp["ld"], grid=w.grid)
+    out = torch.empty_like(ref)
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated(dev)
+    ba.attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, w.d, bias=bias, bias_kind=kind, ld=inp["ld"],
+                             grid=w.grid, out=out)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated(dev) == before          # nothing allocated through torch
+    assert ba.check_device_status() == 0
+    # same kernels, same staging: identical bits
+    assert torch.equal(out, ref)
+    gh, gw = w.grid
+    orc = O.forward(inp["q"], inp["k"], inp["v"], kind, inp["bias"], inp["ld"], gh, gw)["out"]
+    err = np.abs(out.cpu().numpy().astype(np.float64) - orc)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3
