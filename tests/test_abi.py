@@ -87,19 +87,27 @@ def test_bad_dtypes_and_bias_rejected(lib):
     assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, 2, None) == 1
 
 
+def _staged(B, H, N, d, general_relpos=False, keys=128):
+    """Staged key side: tiles of +-1 operand bytes for `keys` keys, then the
+    key scales (and for the general rel-pos bias the key offsets).  A dense
+    bias with B >= 2 runs the paired kernel, whose tiles hold 64 keys."""
+    dpad = 32 * ((d + 31) // 32)
+    tile = keys * dpad + keys * 4 + (keys * 4 if general_relpos else 0)
+    return B * H * ((N + keys - 1) // keys) * tile
+
+
 def test_workspace_size_query(lib):
-    """Size of the staged key side: 64-key tiles of +-1 operand bytes plus key
-    scales (plus key offsets for the general rel-pos bias), and for a rel-pos
-    grid width that is a multiple of 128 four shifted copies of every
-    reversed table row."""
+    """Workspace = staged key tiles, and for a rel-pos grid width that is a
+    multiple of 128 four shifted copies of every reversed table row."""
     ws = lib.ba_attention_workspace_bytes
-    tiles = 16384 // 64
-    kst = 4 * 12 * tiles * (64 * 64 + 64 * 4)
     rps = 12 * (2 * 128 - 1) * 4 * (2 * 128) * 4
+    kst = _staged(4, 12, 16384, 64)
+    assert kst % 256 == 0
     assert ws(4, 12, 16384, 64, 2, 128, 128) == kst + rps
     assert ws(4, 12, 16384, 64, 0, 0, 0) == kst
-    assert ws(32, 12, 577, 64, 1, 0, 0) == 32 * 12 * 10 * (64 * 64 + 256)
-    assert ws(2, 2, 300, 72, 2, 15, 20) == 2 * 2 * 5 * (64 * 96 + 256 + 256)   # general rel-pos: offsets too
+    assert ws(32, 12, 577, 64, 1, 0, 0) == _staged(32, 12, 577, 64, keys=64)
+    assert ws(1, 3, 197, 64, 1, 0, 0) == _staged(1, 3, 197, 64)              # B = 1: nothing to pair
+    assert ws(2, 2, 300, 72, 2, 15, 20) == _staged(2, 2, 300, 72, general_relpos=True)
     assert ws(0, 1, 8, 64, 0, 0, 0) == -1
     assert ws(1, 1, 8, 64, 2, 3, 3) == -1
     assert ws(1, 1, 8, 64, 7, 0, 0) == -1

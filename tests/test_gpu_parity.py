@@ -5,8 +5,9 @@ bit.  Floating outputs: mu within fp32 summation error; the attention output
 within max-abs 2e-2 and mean-abs 2e-3 of the oracle (exact row max, fp64) on
 unit-scale V -- errors are divided by max(1, std of the value channel) so the
 x8 outlier channels of the DeiT-S workload get the same relative budget.  The
-GPU uses a running row max and fp32 arithmetic, so pq can move by one unit;
-that is what the tolerance covers.
+GPU also takes the exact row maximum (two sweeps over the keys) but computes in
+fp32, so a code sitting on a rounding boundary can move by one unit; that is
+what the tolerance covers.
 """
 import numpy as np
 import pytest
@@ -160,6 +161,11 @@ SMALL = [
     ("d128", 1, 1, 140, 128, "bf16", "none", (0, 0)),
     ("d33", 1, 2, 90, 33, "f32", "dense", (0, 0)),
     ("d1", 1, 1, 40, 1, "f32", "none", (0, 0)),
+    # dense bias with B >= 2: the paired kernel (two batch elements per CTA)
+    ("pair_odd_b", 3, 2, 200, 64, "bf16", "dense", (0, 0)),
+    ("pair_d72", 2, 2, 130, 72, "bf16", "dense", (0, 0)),
+    ("pair_d128", 2, 1, 100, 128, "f32", "dense", (0, 0)),
+    ("pair_d32_n64", 4, 1, 64, 32, "bf16", "dense", (0, 0)),
 ]
 
 
