@@ -31,8 +31,9 @@
 //     loader issues no loads or stores of its own;
 //   * QK runs on tcgen05.mma into three S buffers in TMEM, issued up to two
 //     steps ahead of the softmax; both kinds are exact;
-//   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (the
-//     softmax writes it over the S tile it came from) and s8 V tiles,
+//   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (each
+//     softmax thread writes its codes over the S columns it has already
+//     read) and s8 V tiles,
 //     accumulating in TMEM across all key tiles;
 //   * the softmax pulls its 64 keys of an S tile out of TMEM with one load and does
 //     its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with a 3-input
@@ -276,13 +277,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             for (int u = 0; ok && u < U; ++u) {
                 if (u + LA < U && !(ok = issue_qk(u + LA))) break;
                 if (u >= T) {
-                    // PV: u8 P (first BN / 4 columns of the S buffer) x s8 V, K = 32 keys per product.
+                    // PV: u8 P x s8 V, K = 32 keys per product.  The P codes of
+                    // keys 64 h .. 64 h + 63 sit in columns 64 h .. 64 h + 15 of
+                    // the S buffer.
                     const int t = u - T, b = u % NSB, s = u % S;
                     if (!(ok = mbar_wait(&bars[B_SDONE + b], (u / NSB) & 1, abort_flag))) break;
                     tc_fence_after();
                     const uint32_t a_tmem = tmem + b * BN;
                     for (int kk = 0; kk < BN / 32; ++kk)
-                        mma_ts_i8(tmem + O_COL, a_tmem + kk * 8, dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
+                        mma_ts_i8(tmem + O_COL, a_tmem + (kk >> 1) * KH + (kk & 1) * 8,
+                                  dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
                                   idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&bars[B_EMPTY + u % S]);
@@ -378,8 +382,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                     softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                         nvalid, cq2, neg2, mx, l2, pw);
                 // The u8 codes of these 64 keys go back into this row's lane of
-                // the S buffer (16 columns): the PV product reads them from TMEM.
-                tmem_st16(s_col + hf * (KH / 4) + lane_base, pw);
+                // the S buffer, over the first 16 columns of this thread's own
+                // half (already read; the other half's S columns are never
+                // written here): the PV product reads them from TMEM.
+                tmem_st16(s_col + hf * KH + lane_base, pw);
                 tmem_wait_st();
             }
             tc_fence_before();
