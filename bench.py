@@ -36,7 +36,18 @@ from bit_qk_attention_ba_b200.workloads import BIAS_KIND, WORKLOADS, make_inputs
 
 METRIC = "binary attention effective TOPS (4*B*H*N^2*d per step)"
 L2_BYTES = 126 * 2 ** 20
-ATTN_SRC = os.path.join(ROOT, "bit_qk_attention_ba_b200", "csrc", "ba_attn_tc.cu")
+CSRC = os.path.join(ROOT, "bit_qk_attention_ba_b200", "csrc")
+
+
+def attn_kernel(w, variant):
+    """The fused attention kernel a workload runs, and its source file: the
+    CUDA-core kernel for the popcount variant; for a dense bias shared over a
+    batch of two or more, the paired tensor-core kernel; else the 128-key one."""
+    if variant == 1:
+        return "attn_simt_kernel", os.path.join(CSRC, "ba_attn_simt.cu")
+    if w.bias == "dense" and w.B >= 2:
+        return "attn_pair_kernel", os.path.join(CSRC, "ba_attn_tc_pair.cu")
+    return "attn_tc_kernel", os.path.join(CSRC, "ba_attn_tc.cu")
 
 
 # ------------------------------------------------------------------ helpers
@@ -70,10 +81,10 @@ def source_hash(path):
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
 
-def recorded_traffic(kernel_tag, workload):
+def recorded_traffic(kernel, src, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel_tag, workload))
+    p = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel, workload))
     if not os.path.exists(p):
         return None
     vals = {}
@@ -81,7 +92,7 @@ def recorded_traffic(kernel_tag, workload):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_sha256_16") != source_hash(ATTN_SRC):
+    if vals.get("source_sha256_16") != source_hash(src):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -299,7 +310,11 @@ def run_ours(args, w, rank, local_rank, world):
     else:
         roof = {"bound": "hbm", "achieved": abytes / attn_t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic("attn_tc", w.name)
+    kname, ksrc = attn_kernel(w, args.variant)
+    roof["kernel"] = kname
+    roof["traffic"] = recorded_traffic(kname, ksrc, w.name)
+    # CUDA events bracket the whole ba_attention_fwd call: the key staging
+    # pre-passes plus the fused kernel (the staging is the small remainder).
     roof["kernel_us"] = attn_t * 1e6
     roof["peak_source"] = ("int8 = 2 x measured sustained bf16 (%s)" % pk["src"]) if roof["bound"] == "tensor" \
         else "measured HBM copy (%s)" % pk["src"]
