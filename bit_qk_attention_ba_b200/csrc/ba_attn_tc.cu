@@ -201,12 +201,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                                         (BIAS == BA_BIAS_DENSE ? 4 * 16384u : 0u);
             const uint32_t v_bytes = (uint32_t)(2 * p.dv * 64);
             int issued = 0;
-            for (int u = 0; u < U; ++u) {
-                const int s = u % S;
+            int r_s = 0;                           // stage of step u = u % S
+            uint32_t r_p = 0;                      // (u / S) & 1
+            for (int u = 0; u < U; ++u, ring_next(r_s, r_p, S)) {
+                const int s = r_s;
                 const bool pass_b = u >= T;
                 const int t = pass_b ? u - T : u;
                 const int j0 = t * BN;
-                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], (u / S - 1) & 1, abort_flag)) {
+                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag)) {
                     fail(abort_flag, p.status, kStatusTimeoutProducer);
                     break;
                 }
@@ -258,30 +260,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             // the step that used it last (its PV, issued earlier, reads P
             // before this product overwrites it: one thread's tcgen05 ops run
             // in order).
+            // Stage and S buffer of the next QK (issued for steps in order):
+            // slot = step % ring size, parity = (step / ring size) & 1.
+            int q_s = 0, q_b = 0;
+            uint32_t q_sp = 0, q_bp = 0;
             auto issue_qk = [&](int u) -> bool {
-                const int s = u % S, b = u % NSB;
-                if (!mbar_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag)) return false;
-                if (u >= NSB && !mbar_wait(&bars[B_SDONE + b], (u / NSB - 1) & 1, abort_flag)) return false;
+                const int s = q_s, b = q_b;
+                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
+                if (u >= NSB && !mbar_wait(&bars[B_SDONE + b], q_bp ^ 1u, abort_flag)) return false;
                 tc_fence_after();
                 const uint64_t dk = dk0 + s * k_step;
                 const uint32_t d_tmem = tmem + b * BN;
                 for (int kk = 0; kk < kq; ++kk)
                     mma_ss<QK>(d_tmem, dq0 + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
                 mma_commit(&bars[B_SFULL + b]);
+                ring_next(q_s, q_sp, S);
+                ring_next(q_b, q_bp, NSB);
                 return true;
             };
             // QK runs LA steps ahead: two when four stages hold the key tiles
             // of the steps in flight, else one.
             const int LA = (S >= 4) ? 2 : 1;
             for (int u = 0; ok && u < LA && u < U; ++u) ok = issue_qk(u);
-            for (int u = 0; ok && u < U; ++u) {
+            int p_s = 0, p_b = 0;                  // stage and S buffer of step u
+            uint32_t p_sp = 0, p_bp = 0;
+            for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S), ring_next(p_b, p_bp, NSB)) {
                 if (u + LA < U && !(ok = issue_qk(u + LA))) break;
                 if (u >= T) {
                     // PV: u8 P x s8 V, K = 32 keys per product.  The P codes of
                     // keys 64 h .. 64 h + 63 sit in columns 64 h .. 64 h + 15 of
                     // the S buffer.
-                    const int t = u - T, b = u % NSB, s = u % S;
-                    if (!(ok = mbar_wait(&bars[B_SDONE + b], (u / NSB) & 1, abort_flag))) break;
+                    const int t = u - T, b = p_b, s = p_s;
+                    if (!(ok = mbar_wait(&bars[B_SDONE + b], p_bp, abort_flag))) break;
                     tc_fence_after();
                     const uint32_t a_tmem = tmem + b * BN;
                     for (int kk = 0; kk < BN / 32; ++kk)
@@ -289,7 +299,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                                   dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
                                   idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&bars[B_EMPTY + u % S]);
+                mma_commit(&bars[B_EMPTY + p_s]);
             }
             if (ok) mma_commit(&bars[B_OREADY]);
             if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
@@ -343,13 +353,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
         uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         uint64_t neg2 = 0;
         bool ok = true;
-        for (int u = 0; u < U; ++u) {
-            const int s = u % S, b = u % NSB;
+        int r_s = 0, r_b = 0;                         // stage and S buffer of step u
+        uint32_t r_sp = 0, r_bp = 0;
+        for (int u = 0; u < U; ++u, ring_next(r_s, r_sp, S), ring_next(r_b, r_bp, NSB)) {
+            const int s = r_s, b = r_b;
             const bool pass_b = u >= T;
             const int t = pass_b ? u - T : u;
             const int jh = t * BN + hf * KH;          // first key of this thread's half
-            ok = warp_wait(&bars[B_SFULL + b], (u / NSB) & 1, abort_flag) &&
-                 warp_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag);
+            ok = warp_wait(&bars[B_SFULL + b], r_bp, abort_flag) &&
+                 warp_wait(&bars[B_FULL + s], r_sp, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const bool ragged = jh + KH > N;
@@ -430,11 +442,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 uint32_t acc[16];
                 tmem_ld16(tmem + O_COL + c + lane_base, acc);
                 tmem_wait_ld();
-                if (row_ok) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c + e < p.d) store1<OutT>(dst + c + e, __int2float_rn((int)acc[e]) * __ldg(svp + c + e) * inv);
-                }
+                if (row_ok) store_out16<OutT>(dst + c, acc, svp + c, inv, min(16, p.d - c));
             }
         }
     }
@@ -598,7 +606,8 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     const int dv = dv_of(d);
     const int64_t ldv = round_up64(N, 16);
     const int vb = kernel_bias(bias_kind, gw);
-    const bool f8 = variant != BA_QK_TC_I8;
+    // BA_QK_AUTO takes kind::i8 (the faster of the two on B200).
+    const bool f8 = variant == BA_QK_TC_F8;
 
     CUtensorMap tv, tb;
     memset(&tv, 0, sizeof(tv));

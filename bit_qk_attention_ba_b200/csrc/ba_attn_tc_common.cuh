@@ -94,9 +94,51 @@ __device__ __forceinline__ void fail(volatile int* abort_flag, unsigned* status,
     atomicOr(status, bit);
 }
 
+// Advance a running step index i in a ring of n slots, kept as slot = i % n
+// and parity = (i / n) & 1 (no division per step).
+__device__ __forceinline__ void ring_next(int& slot, uint32_t& parity, int n)
+{
+    if (++slot == n) {
+        slot = 0;
+        parity ^= 1u;
+    }
+}
+
 template <typename OutT> __device__ __forceinline__ void store1(OutT* p, float v);
 template <> __device__ __forceinline__ void store1<float>(float* p, float v) { *p = v; }
 template <> __device__ __forceinline__ void store1<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Epilogue for 16 output channels of one row: o_c = sv_c * acc_c * inv for
+// the first n (<= 16) of them, stored as two (bf16) or four (fp32) 16-byte
+// vectors when all 16 are valid and dst is 16-byte aligned, else one by one.
+template <typename OutT>
+__device__ __forceinline__ void store_out16(OutT* dst, const uint32_t (&acc)[16], const float* svp, float inv, int n)
+{
+    float o[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) o[e] = (e < n) ? __int2float_rn((int)acc[e]) * __ldg(svp + e) * inv : 0.f;
+    if (n == 16 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+        if constexpr (sizeof(OutT) == 2) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * e], o[2 * e + 1]);
+                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (e < n) store1<OutT>(dst + e, o[e]);
+    }
+}
 
 // 64 keys of one row: S = z * mu_k * cq + b (Key design 2) on packed
 // pairs, then either the row maximum (pass A) or P~ = exp(S - m), the row sum

@@ -156,12 +156,14 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
             const uint32_t step_bytes = KVG * L.tile + 2 * 16384u;
             const uint32_t v_bytes = (uint32_t)(KVG * p.dv * BN);
             int issued = 0;
-            for (int u = 0; u < U; ++u) {
-                const int s = u % S;
+            int r_s = 0;                           // stage of step u = u % S
+            uint32_t r_p = 0;                      // (u / S) & 1
+            for (int u = 0; u < U; ++u, ring_next(r_s, r_p, S)) {
+                const int s = r_s;
                 const bool pass_b = u >= T;
                 const int t = pass_b ? u - T : u;
                 const int j0 = t * BN;
-                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], (u / S - 1) & 1, abort_flag)) {
+                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag)) {
                     fail(abort_flag, p.status, kStatusTimeoutProducer);
                     break;
                 }
@@ -200,9 +202,13 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
             const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
             const uint32_t q_step = L.q_bytes >> 4, v_step = L.v_bytes >> 4;
             const int kq = p.dpad / 32;
+            // Stage of the next QK (issued for steps in order): slot = step % S,
+            // parity = (step / S) & 1.
+            int q_s = 0;
+            uint32_t q_sp = 0;
             auto issue_qk = [&](int u) -> bool {
-                const int s = u % S, buf = u & 1;
-                if (!mbar_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag)) return false;
+                const int s = q_s, buf = u & 1;
+                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
                 for (int g = 0; g < NG; ++g)
                     if (u >= 2 && !mbar_wait(&bars[B_SDONE + 2 * g + buf], ((u >> 1) - 1) & 1, abort_flag))
                         return false;
@@ -215,14 +221,17 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                         mma_ss<QK>(d_tmem, dq + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
                     mma_commit(&bars[B_SFULL + 2 * g + buf]);
                 }
+                ring_next(q_s, q_sp, S);
                 return true;
             };
             if (ok) ok = issue_qk(0);
-            for (int u = 0; ok && u < U; ++u) {
+            int p_s = 0;                           // stage of step u
+            uint32_t p_sp = 0;
+            for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S)) {
                 if (u + 1 < U && !(ok = issue_qk(u + 1))) break;
                 if (u >= T) {
                     // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
-                    const int t = u - T, buf = u & 1, s = u % S;
+                    const int t = u - T, buf = u & 1, s = p_s;
                     for (int g = 0; g < NG && ok; ++g)
                         ok = mbar_wait(&bars[B_SDONE + 2 * g + buf], (u >> 1) & 1, abort_flag);
                     if (!ok) break;
@@ -235,7 +244,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                                       (t > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(&bars[B_EMPTY + u % S]);
+                mma_commit(&bars[B_EMPTY + p_s]);
             }
             if (ok) mma_commit(&bars[B_OREADY]);
             if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
@@ -279,13 +288,15 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         uint64_t neg2 = 0;
         bool ok = true;
-        for (int u = 0; u < U; ++u) {
-            const int s = u % S, buf = u & 1;
+        int r_s = 0;                                  // stage of step u
+        uint32_t r_sp = 0;
+        for (int u = 0; u < U; ++u, ring_next(r_s, r_sp, S)) {
+            const int s = r_s, buf = u & 1;
             const bool pass_b = u >= T;
             const int t = pass_b ? u - T : u;
             const int j0 = t * BN;
             ok = warp_wait(&bars[B_SFULL + 2 * g + buf], (u >> 1) & 1, abort_flag) &&
-                 warp_wait(&bars[B_FULL + s], (u / S) & 1, abort_flag);
+                 warp_wait(&bars[B_FULL + s], r_sp, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const bool ragged = j0 + BN > N;
@@ -343,11 +354,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                 uint32_t acc[16];
                 tmem_ld16(tmem + 256 + 128 * g + c + lane_base, acc);
                 tmem_wait_ld();
-                if (row_ok) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c + e < p.d) store1<OutT>(dst + c + e, __int2float_rn((int)acc[e]) * __ldg(svp + c + e) * inv);
-                }
+                if (row_ok) store_out16<OutT>(dst + c, acc, svp + c, inv, min(16, p.d - c));
             }
         }
     }

@@ -6,10 +6,16 @@
 // division), code = round-half-even(v / scale) (IEEE fp32 division), clamped
 // to +-127.
 //
-// Three launches, no scratch memory: (1) column absmax folded into the sv
-// output with atomicMax on the (non-negative) float bit patterns, (2)
-// quantise a tile of keys and write it transposed into the channel-major
-// [B, H, d, ldv] code layout, (3) turn the stored absmax into the scale.
+// When all N keys of one (batch, head) fit in shared memory (the ViT / DiT
+// shapes), one launch does everything with one read of V: one CTA per (b, h)
+// stages the [N, d] block, takes the channel absmax, writes the scales and
+// the codes channel-major.  Otherwise three launches, no scratch memory: (1)
+// column absmax folded into the sv output with atomicMax on the
+// (non-negative) float bit patterns, (2) quantise a tile of keys and write it
+// transposed into the channel-major [B, H, d, ldv] code layout, (3) turn the
+// stored absmax into the scale.  In both, codes are transposed through
+// shared memory rows whose stride is an odd number of 4-byte words, so the
+// byte writes of a warp (consecutive channels) land in distinct banks.
 #include "ba_common.cuh"
 
 namespace ba {
@@ -51,6 +57,22 @@ vabsmax_kernel(const T* __restrict__ v, int N, int d, int rows_per_cta, unsigned
         if (red[c]) atomicMax(&amax[bh * d + c], red[c]);
 }
 
+// code = clamp(round_half_even(fl32(x / s)), -127, 127); 0 for an all-zero channel.
+__device__ __forceinline__ uint32_t vcode(float x, float s)
+{
+    if (s == 0.f) return 0u;
+    int q = __float2int_rn(__fdiv_rn(x, s));
+    q = max(-127, min(127, q));
+    return (uint32_t)(q & 0xFF);
+}
+
+// 16 codes of channel row `row` (4-byte aligned, in shared memory) -> 16 bytes of vq.
+__device__ __forceinline__ void store_codes16(int8_t* dst, const uint8_t* row)
+{
+    const uint32_t* q4 = reinterpret_cast<const uint32_t*>(row);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+}
+
 // Tile of 64 keys of one (b, h): quantise and store channel-major.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -58,8 +80,9 @@ vquant_kernel(const T* __restrict__ v, int N, int d, int64_t ldv,
               const unsigned* __restrict__ amax, int8_t* __restrict__ vq)
 {
     constexpr int KT = 64;
+    constexpr int QS = KT + 4;          // code row stride: 17 words
     __shared__ float scale[128];
-    __shared__ __align__(16) int8_t qt[128][KT];
+    __shared__ __align__(16) uint8_t qt[128 * QS];
     const int64_t bh = blockIdx.y;
     const int j0 = blockIdx.x * KT;
     for (int c = threadIdx.x; c < d; c += blockDim.x)
@@ -68,25 +91,61 @@ vquant_kernel(const T* __restrict__ v, int N, int d, int64_t ldv,
     for (int idx = threadIdx.x; idx < KT * d; idx += blockDim.x) {
         const int j = idx / d, c = idx - j * d;
         const int key = j0 + j;
-        int q = 0;
-        if (key < N) {
-            const float s = scale[c];
-            if (s != 0.f) {
-                const float r = __fdiv_rn(to_f32<T>(v[(bh * N + key) * d + c]), s);
-                q = __float2int_rn(r);
-                q = max(-127, min(127, q));
-            }
-        }
-        qt[c][j] = (int8_t)q;
+        qt[c * QS + j] = (uint8_t)((key < N) ? vcode(to_f32<T>(v[(bh * N + key) * d + c]), scale[c]) : 0u);
     }
     __syncthreads();
-    const int groups = KT / 16;
-    for (int idx = threadIdx.x; idx < d * groups; idx += blockDim.x) {
-        const int c = idx / groups, g = idx - c * groups;
+    for (int idx = threadIdx.x; idx < d * (KT / 16); idx += blockDim.x) {
+        const int c = idx >> 2, g = idx & 3;
         const int64_t col = (int64_t)j0 + g * 16;
-        if (col < ldv)
-            *reinterpret_cast<uint4*>(vq + (bh * d + c) * ldv + col) =
-                *reinterpret_cast<const uint4*>(&qt[c][g * 16]);
+        if (col < ldv) store_codes16(vq + (bh * d + c) * ldv + col, qt + c * QS + g * 16);
+    }
+}
+
+// All N keys of one (b, h) in shared memory (tile [N][d] of V, then the codes
+// [d][ldv + 4]): absmax, scale and codes from a single read of V.
+template <typename T>
+__global__ void __launch_bounds__(512)
+vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* __restrict__ vq,
+                    float* __restrict__ sv)
+{
+    extern __shared__ __align__(16) uint8_t sm_raw[];
+    __shared__ unsigned amax[128];
+    __shared__ float scale[128];
+    T* tile = reinterpret_cast<T*>(sm_raw);
+    const int64_t tile_bytes = (int64_t)N * d * sizeof(T);
+    const int qs = (int)ldv + 4;        // odd number of 4-byte words (ldv % 16 == 0)
+    uint8_t* qt = sm_raw + tile_bytes;
+    const int64_t bh = blockIdx.x;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const uint4* src = reinterpret_cast<const uint4*>(v + bh * N * d);
+    for (int64_t i = tid; i < tile_bytes / 16; i += nt) reinterpret_cast<uint4*>(tile)[i] = __ldg(src + i);
+    for (int c = tid; c < d; c += nt) amax[c] = 0u;
+    __syncthreads();
+    const int rows_par = nt / d;
+    if (tid < rows_par * d) {
+        const int c = tid % d;
+        float m = 0.f;
+        for (int r = tid / d; r < N; r += rows_par) m = fmaxf(m, fabsf(to_f32<T>(tile[r * d + c])));
+        atomicMax(&amax[c], __float_as_uint(m));
+    }
+    __syncthreads();
+    for (int c = tid; c < d; c += nt) {
+        const float s = __fdiv_rn(__uint_as_float(amax[c]), 127.0f);
+        scale[c] = s;
+        sv[bh * d + c] = s;
+    }
+    __syncthreads();
+    // ldv * d is below 2^17 here (the block fits in shared memory): 32-bit indices.
+    const int n_codes = (int)ldv * d;
+    for (int idx = tid; idx < n_codes; idx += nt) {
+        const int r = idx / d, c = idx - r * d;
+        qt[c * qs + r] = (uint8_t)((r < N) ? vcode(to_f32<T>(tile[r * d + c]), scale[c]) : 0u);
+    }
+    __syncthreads();
+    const int g16 = (int)(ldv / 16);
+    for (int idx = tid; idx < d * g16; idx += nt) {
+        const int c = idx / g16, g = idx - c * g16;
+        store_codes16(vq + (bh * d + c) * ldv + 16 * g, qt + c * qs + 16 * g);
     }
 }
 
@@ -103,6 +162,15 @@ static cudaError_t launch_quant_v_t(const void* v, int B, int H, int N, int d, i
     const T* vp = static_cast<const T*>(v);
     const int64_t BH = (int64_t)B * H;
     const int64_t ldv = round_up64(N, 16);
+    // Single pass when one (b, h) block of V and its codes fit in shared memory.
+    const int64_t small_smem = (int64_t)N * d * sizeof(T) + (int64_t)d * (ldv + 4);
+    if ((d * sizeof(T)) % 16 == 0 && aligned(v, 16) && small_smem <= 200 * 1024) {
+        auto k = vquant_small_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem);
+        if (e != cudaSuccess) return e;
+        k<<<(unsigned)BH, 512, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv);
+        return cudaGetLastError();
+    }
     cudaError_t e = cudaMemsetAsync(sv, 0, sizeof(float) * BH * d, st);
     if (e != cudaSuccess) return e;
     constexpr int E = 16 / sizeof(T);

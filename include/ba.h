@@ -56,7 +56,7 @@ typedef enum {
 
 /* How the binary Q.K contraction runs inside ba_attention_fwd_variant. */
 typedef enum {
-    BA_QK_AUTO = 0,        /* the fastest path this build has for the shape */
+    BA_QK_AUTO = 0,        /* the fastest path this build has for the shape (tcgen05 kind::i8) */
     BA_QK_POPC = 1,        /* CUDA cores: XOR + popcount on 32-bit words */
     BA_QK_TC_I8 = 3,       /* tcgen05 kind::i8, +-1 int8 operands, s32 in TMEM */
     BA_QK_TC_F8 = 4        /* tcgen05 kind::f8f6f4, +-1 e4m3 operands, f32 in TMEM */
