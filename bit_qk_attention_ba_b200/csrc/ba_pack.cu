@@ -68,6 +68,42 @@ pack_vec_kernel(const T* __restrict__ x, int64_t tokens, int d,
     }
 }
 
+// One thread per token for the common head sizes: the token's NV 16-byte
+// vectors are loaded at once (NV loads in flight per thread, no shuffles),
+// its sign bits and |x| sum built in registers in channel order.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256)
+pack_row_kernel(const T* __restrict__ x, int64_t tokens, int d, uint32_t* __restrict__ bits,
+                float* __restrict__ mu)
+{
+    constexpr int E = 16 / sizeof(T);
+    constexpr int W = (NV * E + 31) / 32;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= tokens) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+    uint4 raw[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) raw[k] = __ldg(src + k);
+    uint32_t w[W];
+#pragma unroll
+    for (int i = 0; i < W; ++i) w[i] = 0u;
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const T* v = reinterpret_cast<const T*>(&raw[k]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int c = k * E + e;
+            const float f = to_f32<T>(v[e]);
+            w[c >> 5] |= (f >= 0.f ? 1u : 0u) << (c & 31);
+            s += fabsf(f);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < W; ++i) bits[t * W + i] = w[i];
+    mu[t] = __fdiv_rn(s, (float)d);
+}
+
 // General fallback: one warp per token, channel c on lane c % 32.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -104,6 +140,15 @@ static cudaError_t launch_pack_t(const void* x, int64_t tokens, int d, uint32_t*
     constexpr int E = 16 / sizeof(T);
     const T* xp = static_cast<const T*>(x);
     const int threads = 256;
+    if (d % E == 0 && aligned(x, 16)) {
+        const unsigned blocks = (unsigned)((tokens + threads - 1) / threads);
+        switch (d / E) {
+#define BA_PACK_ROW(NV) case NV: pack_row_kernel<T, NV><<<blocks, threads, 0, st>>>(xp, tokens, d, bits, mu); return cudaGetLastError();
+            BA_PACK_ROW(2) BA_PACK_ROW(4) BA_PACK_ROW(8) BA_PACK_ROW(9) BA_PACK_ROW(12) BA_PACK_ROW(16)
+#undef BA_PACK_ROW
+            default: break;
+        }
+    }
     if (d % E == 0 && d / E <= 32 && aligned(x, 16)) {
         const int per_warp = 32 / (d / E);
         const int64_t warps = (tokens + per_warp - 1) / per_warp;

@@ -17,6 +17,7 @@
 // shared memory rows whose stride is an odd number of 4-byte words, so the
 // byte writes of a warp (consecutive channels) land in distinct banks.
 #include "ba_common.cuh"
+#include "ba_sm100.cuh"
 
 namespace ba {
 
@@ -106,7 +107,7 @@ vquant_kernel(const T* __restrict__ v, int N, int d, int64_t ldv,
 template <typename T>
 __global__ void __launch_bounds__(512)
 vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* __restrict__ vq,
-                    float* __restrict__ sv)
+                    float* __restrict__ sv, unsigned* __restrict__ status)
 {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     __shared__ unsigned amax[128];
@@ -115,16 +116,36 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
     const int64_t tile_bytes = (int64_t)N * d * sizeof(T);
     const int qs = (int)ldv + 4;        // odd number of 4-byte words (ldv % 16 == 0)
     uint8_t* qt = sm_raw + tile_bytes;
+    __shared__ __align__(8) uint64_t bar;
     const int64_t bh = blockIdx.x;
     const int tid = threadIdx.x, nt = blockDim.x;
-    const uint4* src = reinterpret_cast<const uint4*>(v + bh * N * d);
-    for (int64_t i = tid; i < tile_bytes / 16; i += nt) reinterpret_cast<uint4*>(tile)[i] = __ldg(src + i);
+    // The whole block comes in with bulk copies (at most 64 KB each) on one
+    // mbarrier; the wait is bounded and a timeout only leaves the codes of this
+    // block unwritten after flagging the device status word.
+    if (tid == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::fence_mbar_init();
+    }
     for (int c = tid; c < d; c += nt) amax[c] = 0u;
     __syncthreads();
+    if (tid == 0) {
+        sm100::mbar_arrive_expect_tx(&bar, (uint32_t)tile_bytes);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(v + bh * N * d);
+        for (int64_t off = 0; off < tile_bytes; off += 65536) {
+            const uint32_t n = (uint32_t)min((int64_t)65536, tile_bytes - off);
+            sm100::bulk_load(sm_raw + off, src + off, n, &bar);
+        }
+    }
+    const bool landed = sm100::mbar_wait(&bar, 0, nullptr);
+    if (!__syncthreads_and(landed)) {
+        if (tid == 0) atomicOr(status, kStatusTimeoutProducer);
+        return;
+    }
     const int rows_par = nt / d;
     if (tid < rows_par * d) {
         const int c = tid % d;
         float m = 0.f;
+#pragma unroll 4
         for (int r = tid / d; r < N; r += rows_par) m = fmaxf(m, fabsf(to_f32<T>(tile[r * d + c])));
         atomicMax(&amax[c], __float_as_uint(m));
     }
@@ -137,6 +158,7 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
     __syncthreads();
     // ldv * d is below 2^17 here (the block fits in shared memory): 32-bit indices.
     const int n_codes = (int)ldv * d;
+#pragma unroll 4
     for (int idx = tid; idx < n_codes; idx += nt) {
         const int r = idx / d, c = idx - r * d;
         qt[c * qs + r] = (uint8_t)((r < N) ? vcode(to_f32<T>(tile[r * d + c]), scale[c]) : 0u);
@@ -168,7 +190,9 @@ static cudaError_t launch_quant_v_t(const void* v, int B, int H, int N, int d, i
         auto k = vquant_small_kernel<T>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem);
         if (e != cudaSuccess) return e;
-        k<<<(unsigned)BH, 512, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv);
+        unsigned* status = device_status_ptr();
+        if (!status) return cudaErrorInvalidDevice;
+        k<<<(unsigned)BH, 512, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv, status);
         return cudaGetLastError();
     }
     cudaError_t e = cudaMemsetAsync(sv, 0, sizeof(float) * BH * d, st);
