@@ -59,10 +59,19 @@ vabsmax_kernel(const T* __restrict__ v, int N, int d, int rows_per_cta, unsigned
 }
 
 // code = clamp(round_half_even(fl32(x / s)), -127, 127); 0 for an all-zero channel.
-__device__ __forceinline__ uint32_t vcode(float x, float s)
+// rs = fl32(1 / s).  Here |x| <= 127 s, so t = fl32(x * rs) is within 3e-5 of
+// x / s and fl32(x / s) within 8e-6 of it: when t is more than 1e-4 away from
+// a rounding boundary (k + 1/2), both round to the same integer, and the code
+// is rint(t); otherwise the IEEE quotient is formed and rounded.  Either way
+// the result equals rounding fl32(x / s).
+__device__ __forceinline__ uint32_t vcode(float x, float s, float rs)
 {
     if (s == 0.f) return 0u;
-    int q = __float2int_rn(__fdiv_rn(x, s));
+    const float t = x * rs;
+    const float k = (t + 12582912.f) - 12582912.f;     // round-half-even of t (|t| < 2^22)
+    int q;
+    if (0.5f - fabsf(t - k) > 1e-4f) q = (int)k;
+    else q = __float2int_rn(__fdiv_rn(x, s));
     q = max(-127, min(127, q));
     return (uint32_t)(q & 0xFF);
 }
@@ -82,17 +91,23 @@ vquant_kernel(const T* __restrict__ v, int N, int d, int64_t ldv,
 {
     constexpr int KT = 64;
     constexpr int QS = KT + 4;          // code row stride: 17 words
-    __shared__ float scale[128];
+    __shared__ float scale[128], rscale[128];
     __shared__ __align__(16) uint8_t qt[128 * QS];
     const int64_t bh = blockIdx.y;
     const int j0 = blockIdx.x * KT;
-    for (int c = threadIdx.x; c < d; c += blockDim.x)
-        scale[c] = __fdiv_rn(__uint_as_float(amax[bh * d + c]), 127.0f);
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        const float sc = __fdiv_rn(__uint_as_float(amax[bh * d + c]), 127.0f);
+        scale[c] = sc;
+        rscale[c] = __frcp_rn(sc);
+    }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < KT * d; idx += blockDim.x) {
-        const int j = idx / d, c = idx - j * d;
+    // (key j, channel c) with c fastest, stepped without a division per element.
+    const int nt = blockDim.x, dj = nt / d, dc = nt - dj * d;
+    int j = threadIdx.x / d, c = threadIdx.x - j * d;
+    for (; j < KT; j += dj, c += dc) {
+        if (c >= d) { c -= d; ++j; if (j >= KT) break; }
         const int key = j0 + j;
-        qt[c * QS + j] = (uint8_t)((key < N) ? vcode(to_f32<T>(v[(bh * N + key) * d + c]), scale[c]) : 0u);
+        qt[c * QS + j] = (uint8_t)((key < N) ? vcode(to_f32<T>(v[(bh * N + key) * d + c]), scale[c], rscale[c]) : 0u);
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < d * (KT / 16); idx += blockDim.x) {
@@ -111,7 +126,7 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
 {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     __shared__ unsigned amax[128];
-    __shared__ float scale[128];
+    __shared__ float scale[128], rscale[128];
     T* tile = reinterpret_cast<T*>(sm_raw);
     const int64_t tile_bytes = (int64_t)N * d * sizeof(T);
     const int qs = (int)ldv + 4;        // odd number of 4-byte words (ldv % 16 == 0)
@@ -153,15 +168,19 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
     for (int c = tid; c < d; c += nt) {
         const float s = __fdiv_rn(__uint_as_float(amax[c]), 127.0f);
         scale[c] = s;
+        rscale[c] = __frcp_rn(s);
         sv[bh * d + c] = s;
     }
     __syncthreads();
-    // ldv * d is below 2^17 here (the block fits in shared memory): 32-bit indices.
-    const int n_codes = (int)ldv * d;
+    // (key r, channel c) with c fastest, stepped without a division per element.
+    {
+        const int dr = nt / d, dc = nt - dr * d, rows = (int)ldv;
+        int r = tid / d, c = tid - r * d;
 #pragma unroll 4
-    for (int idx = tid; idx < n_codes; idx += nt) {
-        const int r = idx / d, c = idx - r * d;
-        qt[c * qs + r] = (uint8_t)((r < N) ? vcode(to_f32<T>(tile[r * d + c]), scale[c]) : 0u);
+        for (; r < rows; r += dr, c += dc) {
+            if (c >= d) { c -= d; ++r; if (r >= rows) break; }
+            qt[c * qs + r] = (uint8_t)((r < N) ? vcode(to_f32<T>(tile[r * d + c]), scale[c], rscale[c]) : 0u);
+        }
     }
     __syncthreads();
     const int g16 = (int)(ldv / 16);

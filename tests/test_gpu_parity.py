@@ -101,6 +101,30 @@ def test_pack_and_quant_full_size(name):
     assert not vq[..., w.N:].any()
 
 
+@pytest.mark.parametrize("N", [300, 5000])
+def test_quant_codes_at_rounding_boundaries(N):
+    """V values placed on and next to the code boundaries x / s = k + 1/2
+    (ties included) for several channel scales s; the codes must match the
+    oracle's IEEE fp32 division and round-half-even bit for bit.  N = 300 runs
+    the single-pass quantiser, N = 5000 the tiled one."""
+    rng = np.random.default_rng(7)
+    d = 64
+    absmax = np.array([127.0, 12.7, 38.1, 1.0, 0.3, 1e-3, 5e4, 3.0] * 8, np.float32)
+    s = (absmax / np.float32(127.0)).astype(np.float32)
+    k = rng.integers(-127, 127, size=(N, d)).astype(np.float32)
+    delta = rng.choice(np.array([0.0, 1e-7, -1e-7, 1e-6, -1e-6, 1e-5, -1e-5, 1e-4, -1e-4, 3e-3], np.float32),
+                       size=(N, d))
+    v = ((k + np.float32(0.5) + delta) * s).astype(np.float32)
+    v[0] = absmax                      # pin each channel's absmax
+    v = np.clip(v, -absmax, absmax).astype(np.float32)
+    vt = torch.from_numpy(v.reshape(1, 1, N, d)).to(DEV).contiguous()
+    vq, sv = ba.quant_v(vt)
+    torch.cuda.synchronize()
+    ovq, osv = O.quant_v(v.reshape(1, N, d))
+    np.testing.assert_array_equal(sv.cpu().numpy().reshape(osv.shape), osv)
+    np.testing.assert_array_equal(_vq_natural(vq, N), ovq)
+
+
 @pytest.mark.parametrize("d", [1, 31, 33, 72, 96, 128])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_pack_and_quant_odd_d(d, dtype):
