@@ -1,6 +1,10 @@
 // ba_attn_tc_pair.cu -- the tensor-core attention for a dense bias shared
-// over the batch: one CTA takes the same 128 query rows of two batch elements
-// (two row groups), so one staged bias tile serves both.
+// over the batch: a work tile is the same 128 query rows of two batch
+// elements (two row groups), so one staged bias tile serves both.  The kernel
+// is persistent (one CTA per SM walks tiles blockIdx.x, + gridDim.x, ...): the
+// loader and the MMA thread start the next tile while the softmax warps are
+// still in the previous tile's epilogue, and no CTA launch, TMEM allocation or
+// pipeline fill is paid per tile.
 //
 // BA notes (paper-notes page "BinaryAttention: One-Bit QK-Attention for
 // Vision and Diffusion Transformers", CVPR 2026): Key designs 1-3 and the
@@ -37,8 +41,9 @@ enum {
     B_EMPTY = B_FULL + MAX_STAGES,   // [stage] stage may be overwritten
     B_SFULL = B_EMPTY + MAX_STAGES,  // [NG][2] S tile in TMEM ready
     B_SDONE = B_SFULL + 2 * NG,      // [NG][2] softmax done with the S buffer (pass B: u8 P written into it)
-    B_OREADY = B_SDONE + 2 * NG,     // every PV finished
-    B_FINAL = B_OREADY + 1,
+    B_OREADY = B_SDONE + 2 * NG,     // every PV of the tile finished (one phase per tile)
+    B_OFREE = B_OREADY + 1,          // the softmax warps read the tile's output accumulators
+    B_FINAL = B_OFREE + 1,
     NUM_BARS
 };
 
@@ -77,19 +82,35 @@ struct Params {
     const float* sv;
     void* out;
     int B, H, N, d, W, dpad, dv, n_tiles, stages;
+    int tiles_x, tiles;      // row blocks per head; work tiles (row block, head, batch pair)
     float q_scale;           // 1 / sqrt(d)
     unsigned* status;
 };
 
-// Which (batch*head, first query row) group g of this CTA covers and whether
-// it exists: batch elements 2z and 2z + 1 of head y, rows 128 x.
-__device__ __forceinline__ void group_coords(const Params& p, int g, int& bh, int& q0, bool& exists)
+// Work tile k = (row block x, head y, batch pair z), x fastest.
+struct TileCoord {
+    int x, y, z;
+};
+__device__ __forceinline__ TileCoord tile_coord(const Params& p, int k)
 {
-    int b = 2 * blockIdx.z + g;
+    TileCoord c;
+    c.x = k % p.tiles_x;
+    const int rest = k / p.tiles_x;
+    c.y = rest % p.H;
+    c.z = rest / p.H;
+    return c;
+}
+
+// Which (batch*head, first query row) group g of a tile covers and whether it
+// exists: batch elements 2z and 2z + 1 of head y, rows 128 x.
+__device__ __forceinline__ void group_coords(const Params& p, const TileCoord& tc, int g, int& bh, int& q0,
+                                             bool& exists)
+{
+    int b = 2 * tc.z + g;
     exists = b < p.B;
     if (!exists) b = p.B - 1;
-    bh = b * p.H + blockIdx.y;
-    q0 = blockIdx.x * BM;
+    bh = b * p.H + tc.y;
+    q0 = tc.x * BM;
 }
 
 template <int QK, typename OutT>
@@ -110,7 +131,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
     const int N = p.N, W = p.W, T = p.n_tiles, U = 2 * T;   // steps: pass A then pass B
     const int S = p.stages;
     const int chunks = p.dpad / 16;
-    const int h = (int)blockIdx.y;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_QREADY], NUM_SOFTMAX_WARPS);
@@ -123,6 +143,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
             mbar_init(&bars[B_SDONE + b], 4);
         }
         mbar_init(&bars[B_OREADY], 1);
+        mbar_init(&bars[B_OFREE], NUM_SOFTMAX_WARPS);
         mbar_init(&bars[B_FINAL], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -147,44 +168,46 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         // in pass B the two V tiles.  All copies complete on the stage's FULL
         // barrier.
         if (lane == 0) {
-            int kvbh0, kvbh1, q0g;
-            {
-                bool ex;
-                group_coords(p, 0, kvbh0, q0g, ex);
-                group_coords(p, 1, kvbh1, q0g, ex);
-            }
             const uint32_t step_bytes = KVG * L.tile + 2 * 16384u;
             const uint32_t v_bytes = (uint32_t)(KVG * p.dv * BN);
-            int issued = 0;
-            int r_s = 0;                           // stage of step u = u % S
-            uint32_t r_p = 0;                      // (u / S) & 1
-            for (int u = 0; u < U; ++u, ring_next(r_s, r_p, S)) {
-                const int s = r_s;
-                const bool pass_b = u >= T;
-                const int t = pass_b ? u - T : u;
-                const int j0 = t * BN;
-                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag)) {
-                    fail(abort_flag, p.status, kStatusTimeoutProducer);
-                    break;
+            int64_t issued = 0, gstep = 0;         // steps issued, all tiles
+            int r_s = 0;                           // stage of the running step = gstep % S
+            uint32_t r_p = 0;                      // (gstep / S) & 1
+            bool ok = true;
+            for (int k = blockIdx.x; ok && k < p.tiles; k += gridDim.x) {
+                const TileCoord tc = tile_coord(p, k);
+                int kvbh0, kvbh1, q0g;
+                bool ex;
+                group_coords(p, tc, 0, kvbh0, q0g, ex);
+                group_coords(p, tc, 1, kvbh1, q0g, ex);
+                for (int u = 0; u < U; ++u, ++gstep, ring_next(r_s, r_p, S)) {
+                    const int s = r_s;
+                    const bool pass_b = u >= T;
+                    const int t = pass_b ? u - T : u;
+                    const int j0 = t * BN;
+                    if (gstep >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag)) {
+                        fail(abort_flag, p.status, kStatusTimeoutProducer);
+                        ok = false;
+                        break;
+                    }
+                    uint64_t* full = &bars[B_FULL + s];
+                    mbar_arrive_expect_tx(full, step_bytes + (pass_b ? v_bytes : 0u));
+                    uint8_t* kdst = smem + L.k + s * L.k_bytes;
+                    bulk_load(kdst, p.kst + ((size_t)kvbh0 * T + t) * L.tile, L.tile, full);
+                    bulk_load(kdst + L.tile, p.kst + ((size_t)kvbh1 * T + t) * L.tile, L.tile, full);
+                    for (int bx = 0; bx < 2; ++bx)
+                        tma_load_3d(smem + L.b + (s * 2 + bx) * 16384, &tm_b, full, j0 + 32 * bx, q0g, tc.y);
+                    if (pass_b) {
+                        tma_load_3d(smem + L.v + (s * KVG) * L.v_bytes, &tm_v, full, j0, 0, kvbh0);
+                        tma_load_3d(smem + L.v + (s * KVG + 1) * L.v_bytes, &tm_v, full, j0, 0, kvbh1);
+                    }
+                    issued = gstep + 1;
                 }
-                uint64_t* full = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(full, step_bytes + (pass_b ? v_bytes : 0u));
-                uint8_t* kdst = smem + L.k + s * L.k_bytes;
-                bulk_load(kdst, p.kst + ((size_t)kvbh0 * T + t) * L.tile, L.tile, full);
-                if (KVG > 1) bulk_load(kdst + L.tile, p.kst + ((size_t)kvbh1 * T + t) * L.tile, L.tile, full);
-                for (int bx = 0; bx < 2; ++bx)
-                        tma_load_3d(smem + L.b + (s * 2 + bx) * 16384, &tm_b, full, j0 + 32 * bx,
-                                    (int)blockIdx.x * BM, h);
-                if (pass_b) {
-                    tma_load_3d(smem + L.v + (s * KVG) * L.v_bytes, &tm_v, full, j0, 0, kvbh0);
-                    if (KVG > 1) tma_load_3d(smem + L.v + (s * KVG + 1) * L.v_bytes, &tm_v, full, j0, 0, kvbh1);
-                }
-                issued = u + 1;
             }
             // On an abort, let copies already issued land before the CTA exits.
             if (*abort_flag)
-                for (int u = (issued > S ? issued - S : 0); u < issued; ++u)
-                    mbar_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
+                for (int64_t w = (issued > S ? issued - S : 0); w < issued; ++w)
+                    mbar_wait(&bars[B_FULL + (int)(w % S)], (uint32_t)((w / S) & 1), nullptr, 100000000ull);
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
@@ -194,7 +217,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                                                     : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
             const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
             const uint32_t sbo_qk = (uint32_t)chunks * 128u;
-            bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag);
             // Descriptors are built once; moving along a buffer only adds to the
             // start-address field (bytes / 16), which never carries out.
             const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
@@ -202,15 +224,15 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
             const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
             const uint32_t q_step = L.q_bytes >> 4, v_step = L.v_bytes >> 4;
             const int kq = p.dpad / 32;
-            // Stage of the next QK (issued for steps in order): slot = step % S,
-            // parity = (step / S) & 1.
-            int q_s = 0;
+            // Steps run on across tiles: the S buffer of global step w is w & 1,
+            // in its use (w >> 1); ring slots and parities are running counters.
+            int q_s = 0;                           // stage of the next QK
             uint32_t q_sp = 0;
-            auto issue_qk = [&](int u) -> bool {
-                const int s = q_s, buf = u & 1;
+            auto issue_qk = [&](int64_t w) -> bool {
+                const int s = q_s, buf = (int)(w & 1);
                 if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
                 for (int g = 0; g < NG; ++g)
-                    if (u >= 2 && !mbar_wait(&bars[B_SDONE + 2 * g + buf], ((u >> 1) - 1) & 1, abort_flag))
+                    if (w >= 2 && !mbar_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)(((w >> 1) - 1) & 1), abort_flag))
                         return false;
                 tc_fence_after();
                 for (int g = 0; g < NG; ++g) {
@@ -224,29 +246,42 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                 ring_next(q_s, q_sp, S);
                 return true;
             };
-            if (ok) ok = issue_qk(0);
-            int p_s = 0;                           // stage of step u
+            bool ok = true;
+            int p_s = 0;                           // stage of the running step
             uint32_t p_sp = 0;
-            for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S)) {
-                if (u + 1 < U && !(ok = issue_qk(u + 1))) break;
-                if (u >= T) {
-                    // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
-                    const int t = u - T, buf = u & 1, s = p_s;
-                    for (int g = 0; g < NG && ok; ++g)
-                        ok = mbar_wait(&bars[B_SDONE + 2 * g + buf], (u >> 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    for (int g = 0; g < NG; ++g) {
-                        const uint64_t dv = dv0 + (s * KVG + g) * v_step;
-                        const uint32_t a_tmem = tmem + (2 * g + buf) * BN;
-                        for (int kk = 0; kk < BN / 32; ++kk)
-                            mma_ts_i8(tmem + 256 + 128 * g, a_tmem + kk * 8, dv + kk * 2, idesc_pv,
-                                      (t > 0 || kk > 0) ? 1u : 0u);
+            int64_t gbase = 0;                     // global index of the tile's first step
+            int kt = 0;                            // tiles done by this CTA
+            for (int k = blockIdx.x; ok && k < p.tiles; k += gridDim.x, ++kt, gbase += U) {
+                // Q of this tile written by the softmax warps.
+                if (!(ok = mbar_wait(&bars[B_QREADY], (uint32_t)(kt & 1), abort_flag))) break;
+                if (!(ok = issue_qk(gbase))) break;
+                for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S)) {
+                    const int64_t w = gbase + u;
+                    if (u + 1 < U && !(ok = issue_qk(w + 1))) break;
+                    if (u >= T) {
+                        // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
+                        const int t = u - T, buf = (int)(w & 1), s = p_s;
+                        // The first PV of a tile overwrites the output accumulators:
+                        // the softmax warps must have read the previous tile's.
+                        if (t == 0 && kt > 0 &&
+                            !(ok = mbar_wait(&bars[B_OFREE], (uint32_t)((kt - 1) & 1), abort_flag)))
+                            break;
+                        for (int g = 0; g < NG && ok; ++g)
+                            ok = mbar_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)((w >> 1) & 1), abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        for (int g = 0; g < NG; ++g) {
+                            const uint64_t dv = dv0 + (s * KVG + g) * v_step;
+                            const uint32_t a_tmem = tmem + (2 * g + buf) * BN;
+                            for (int kk = 0; kk < BN / 32; ++kk)
+                                mma_ts_i8(tmem + 256 + 128 * g, a_tmem + kk * 8, dv + kk * 2, idesc_pv,
+                                          (t > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
+                    mma_commit(&bars[B_EMPTY + p_s]);
                 }
-                mma_commit(&bars[B_EMPTY + p_s]);
+                if (ok) mma_commit(&bars[B_OREADY]);
             }
-            if (ok) mma_commit(&bars[B_OREADY]);
             if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
             // Let every issued MMA finish before TMEM is released.
             mma_commit(&bars[B_FINAL]);
@@ -258,21 +293,21 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         const int g = warp >> 2;                      // row group
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;            // row within the group
-        int bh, q0;
-        bool group_exists;
-        group_coords(p, g, bh, q0, group_exists);
-        const int i = q0 + r;
-        const bool row_ok = group_exists && i < N;
-        const int ie = (i < N) ? i : N - 1;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const int kvx = g;
-
-        // Q operand of this row, padding channels zeroed.
-        {
-            uint8_t* qop = smem + L.q + g * L.q_bytes;
-            const uint32_t* src = p.bq + ((size_t)bh * N + ie) * W;
+        uint8_t* qop = smem + L.q + g * L.q_bytes;
+        // Q operand of this row for tile k, padding channels zeroed.  This
+        // group's QK products of the previous tile have all completed (its last
+        // S tile was waited for), so the operand may be overwritten.
+        auto write_q = [&](int k) {
+            int bh, q0;
+            bool ex;
+            group_coords(p, tile_coord(p, k), g, bh, q0, ex);
+            const int i = q0 + r;
+            const bool rok = ex && i < N;
+            const uint32_t* src = p.bq + ((size_t)bh * N + ((i < N) ? i : N - 1)) * W;
             for (int w = 0; w < W; ++w) {
-                const uint32_t bits = row_ok ? __ldg(src + w) : 0u;
+                const uint32_t bits = rok ? __ldg(src + w) : 0u;
                 const int nvalid = min(32, p.d - 32 * w);
                 const uint32_t vm = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
                 *reinterpret_cast<uint4*>(qop + core_off(r, 2 * w, chunks)) = expand16<QK>(bits & 0xFFFFu, vm & 0xFFFFu);
@@ -281,68 +316,79 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_QREADY]);
-        }
-        const float cq = row_ok ? __ldg(p.muq + (size_t)bh * N + i) * p.q_scale : 0.f;
-        const uint64_t cq2 = f2_pack(cq, cq);
-        float mrow = -INFINITY;
-        uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        uint64_t neg2 = 0;
+        };
         bool ok = true;
-        int r_s = 0;                                  // stage of step u
+        int r_s = 0;                                  // stage of the running step
         uint32_t r_sp = 0;
-        for (int u = 0; u < U; ++u, ring_next(r_s, r_sp, S)) {
-            const int s = r_s, buf = u & 1;
-            const bool pass_b = u >= T;
-            const int t = pass_b ? u - T : u;
-            const int j0 = t * BN;
-            ok = warp_wait(&bars[B_SFULL + 2 * g + buf], (u >> 1) & 1, abort_flag) &&
-                 warp_wait(&bars[B_FULL + s], r_sp, abort_flag);
+        int64_t gbase = 0;                            // global index of the tile's first step
+        int kt = 0;
+        if ((int)blockIdx.x < p.tiles) write_q(blockIdx.x);
+        for (int k = blockIdx.x; ok && k < p.tiles; k += gridDim.x, ++kt, gbase += U) {
+            int bh, q0;
+            bool group_exists;
+            group_coords(p, tile_coord(p, k), g, bh, q0, group_exists);
+            const int i = q0 + r;
+            const bool row_ok = group_exists && i < N;
+            const int ie = (i < N) ? i : N - 1;
+            const float cq = row_ok ? __ldg(p.muq + (size_t)bh * N + i) * p.q_scale : 0.f;
+            const uint64_t cq2 = f2_pack(cq, cq);
+            float mrow = -INFINITY;
+            uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+            uint64_t neg2 = 0;
+            for (int u = 0; u < U; ++u, ring_next(r_s, r_sp, S)) {
+                const int64_t w = gbase + u;
+                const int s = r_s, buf = (int)(w & 1);
+                const bool pass_b = u >= T;
+                const int t = pass_b ? u - T : u;
+                const int j0 = t * BN;
+                ok = warp_wait(&bars[B_SFULL + 2 * g + buf], (uint32_t)((w >> 1) & 1), abort_flag) &&
+                     warp_wait(&bars[B_FULL + s], r_sp, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const bool ragged = j0 + BN > N;
+                const uint8_t* tile_s = smem + L.k + s * L.k_bytes + kvx * L.tile;
+                const float* muk_s = reinterpret_cast<const float*>(tile_s + BN * p.dpad);
+                const uint8_t* bsm_row = smem + L.b + s * 2 * 16384 + r * 128;
+                const int nvalid = N - j0;
+                uint32_t zr[64];
+                tmem_ld64(tmem + (2 * g + buf) * BN + lane_base, zr);
+                tmem_wait_ld();
+                uint32_t pw[16];
+                float mx[2] = {-INFINITY, -INFINITY};
+                if (!pass_b) {
+                    if (ragged)
+                        softmax_tile<QK, BIAS, false, true>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
+                                                            nvalid, cq2, neg2, mx, l2, pw);
+                    else
+                        softmax_tile<QK, BIAS, false, false>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
+                                                             nvalid, cq2, neg2, mx, l2, pw);
+                    mrow = fmax3(mrow, mx[0], mx[1]);
+                } else {
+                    if (ragged)
+                        softmax_tile<QK, BIAS, true, true>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
+                                                           nvalid, cq2, neg2, mx, l2, pw);
+                    else
+                        softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
+                                                            nvalid, cq2, neg2, mx, l2, pw);
+                    // The u8 codes go back into this row's lane of the S buffer: the
+                    // PV product reads them from TMEM.
+                    tmem_st16(tmem + (2 * g + buf) * BN + lane_base, pw);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bars[B_SDONE + 2 * g + buf]);
+                    mbar_arrive(&bars[B_EMPTY + s]);
+                }
+                if (u == T - 1) neg2 = f2_pack(-mrow * LOG2E, -mrow * LOG2E);
+            }
             if (!ok) break;
-            tc_fence_after();
-            const bool ragged = j0 + BN > N;
-            const uint8_t* tile_s = smem + L.k + s * L.k_bytes + kvx * L.tile;
-            const float* muk_s = reinterpret_cast<const float*>(tile_s + BN * p.dpad);
-            const uint8_t* bsm_row = smem + L.b + s * 2 * 16384 + r * 128;
-            const int nvalid = N - j0;
-            uint32_t zr[64];
-            tmem_ld64(tmem + (2 * g + buf) * BN + lane_base, zr);
-            tmem_wait_ld();
-            uint32_t pw[16];
-            float mx[2] = {-INFINITY, -INFINITY};
-            if (!pass_b) {
-                if (ragged)
-                    softmax_tile<QK, BIAS, false, true>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
-                                                        nvalid, cq2, neg2, mx, l2, pw);
-                else
-                    softmax_tile<QK, BIAS, false, false>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
-                                                         nvalid, cq2, neg2, mx, l2, pw);
-                mrow = fmax3(mrow, mx[0], mx[1]);
-            } else {
-                if (ragged)
-                    softmax_tile<QK, BIAS, true, true>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
-                                                       nvalid, cq2, neg2, mx, l2, pw);
-                else
-                    softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, nullptr, nullptr, nullptr, 0,
-                                                        nvalid, cq2, neg2, mx, l2, pw);
-                // The u8 codes go back into this row's lane of the S buffer: the
-                // PV product reads them from TMEM.
-                tmem_st16(tmem + (2 * g + buf) * BN + lane_base, pw);
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[B_SDONE + 2 * g + buf]);
-                mbar_arrive(&bars[B_EMPTY + s]);
-            }
-            if (u == T - 1) neg2 = f2_pack(-mrow * LOG2E, -mrow * LOG2E);
-        }
+            // The next tile's Q goes in now, so its QK products overlap this epilogue.
+            if (k + (int)gridDim.x < p.tiles) write_q(k + gridDim.x);
 
-        // Epilogue: O = sv * acc / (255 l).
-        if (ok) ok = warp_wait(&bars[B_OREADY], 0, abort_flag);
-        if (!ok) {
-            if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutSoftmax);
-        } else {
+            // Epilogue: O = sv * acc / (255 l).
+            if (!(ok = warp_wait(&bars[B_OREADY], (uint32_t)(kt & 1), abort_flag))) break;
             tc_fence_after();
             float la, lb, lc, ld;
             f2_unpack(l2[0], la, lb);
@@ -356,7 +402,12 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
                 tmem_wait_ld();
                 if (row_ok) store_out16<OutT>(dst + c, acc, svp + c, inv, min(16, p.d - c));
             }
+            // The output accumulators may take the next tile's PV products.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_OFREE]);
         }
+        if (!ok && lane == 0) fail(abort_flag, p.status, kStatusTimeoutSoftmax);
     }
 
     tc_fence_before();
@@ -390,7 +441,11 @@ cudaError_t launch_t(const CUtensorMap& tv, const CUtensorMap& tb, const Params&
     auto kern = attn_pair_kernel<QK, OutT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(p.N, BM), p.H, ceil_div(p.B, 2));
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // Persistent: one CTA per SM (each takes all TMEM columns), at most one per tile.
+    const int grid = p.tiles < sms ? p.tiles : sms;
     kern<<<grid, NUM_THREADS, smem, st>>>(tv, tb, p);
     return cudaGetLastError();
 }
@@ -439,6 +494,8 @@ cudaError_t launch_attn_pair(const uint32_t* bq, const float* muq, const uint8_t
     p.bq = bq; p.muq = muq; p.kst = kst; p.sv = sv; p.out = out;
     p.B = B; p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
     p.n_tiles = ceil_div(N, BN);
+    p.tiles_x = ceil_div(N, BM);
+    p.tiles = p.tiles_x * H * ceil_div(B, 2);
     p.stages = pick_stages(d);
     p.q_scale = (float)(1.0 / sqrt((double)d));
     p.status = status;
