@@ -156,13 +156,35 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
         if (tid == 0) atomicOr(status, kStatusTimeoutProducer);
         return;
     }
-    const int rows_par = nt / d;
-    if (tid < rows_par * d) {
-        const int c = tid % d;
-        float m = 0.f;
+    // Each thread owns four consecutive channels (d % 4 == 0 here) and walks
+    // the rows: one 8- or 16-byte shared-memory read per row, the scales in
+    // registers.
+    const int G4 = d / 4;
+    const int dr = nt / G4;
+    const bool active = tid < dr * G4;
+    const int c4 = tid % G4, r0 = tid / G4;
+    auto load4 = [&](int r, float (&x)[4]) {
+        if constexpr (sizeof(T) == 2) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(tile + r * d + 4 * c4);
+            const T* h = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = to_f32<T>(h[e]);
+        } else {
+            const float4 raw = *reinterpret_cast<const float4*>(tile + r * d + 4 * c4);
+            x[0] = raw.x; x[1] = raw.y; x[2] = raw.z; x[3] = raw.w;
+        }
+    };
+    if (active) {
+        float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-        for (int r = tid / d; r < N; r += rows_par) m = fmaxf(m, fabsf(to_f32<T>(tile[r * d + c])));
-        atomicMax(&amax[c], __float_as_uint(m));
+        for (int r = r0; r < N; r += dr) {
+            float x[4];
+            load4(r, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) atomicMax(&amax[4 * c4 + e], __float_as_uint(m[e]));
     }
     __syncthreads();
     for (int c = tid; c < d; c += nt) {
@@ -172,14 +194,22 @@ vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* 
         sv[bh * d + c] = s;
     }
     __syncthreads();
-    // (key r, channel c) with c fastest, stepped without a division per element.
-    {
-        const int dr = nt / d, dc = nt - dr * d, rows = (int)ldv;
-        int r = tid / d, c = tid - r * d;
-#pragma unroll 4
-        for (; r < rows; r += dr, c += dc) {
-            if (c >= d) { c -= d; ++r; if (r >= rows) break; }
-            qt[c * qs + r] = (uint8_t)((r < N) ? vcode(to_f32<T>(tile[r * d + c]), scale[c], rscale[c]) : 0u);
+    if (active) {
+        float sc[4], rs[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sc[e] = scale[4 * c4 + e];
+            rs[e] = rscale[4 * c4 + e];
+        }
+        uint8_t* qrow = qt + (4 * c4) * qs;
+        const int rows = (int)ldv;
+#pragma unroll 2
+        for (int r = r0; r < rows; r += dr) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (r < N) load4(r, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                qrow[e * qs + r] = (uint8_t)((r < N) ? vcode(x[e], sc[e], rs[e]) : 0u);
         }
     }
     __syncthreads();
