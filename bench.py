@@ -177,6 +177,12 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
 
 
+def aggregate_tops(world, ops_per_rank, ms_per_step):
+    """Whole-job effective TOPS: every rank runs its own copy of the workload
+    (replicas, weak scaling), timed by the slowest rank."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def max_over_ranks(x, world, device=None):
     """Max of a float over ranks (identity for one process)."""
     if world <= 1:
@@ -299,7 +305,7 @@ def run_ours(args, w, rank, local_rank, world):
     tc_path = ws is not None and args.variant != NAT.BA_QK_POPC
     fast_rp = kind == NAT.BA_BIAS_RELPOS2D and grid and grid[1] % 128 == 0
     launches_per_step = 5 + (1 + (1 if fast_rp else 0) if tc_path else 0) + 1
-    value = world * ops / (ms * 1e-3) / 1e12
+    value = aggregate_tops(world, ops, ms)
     pk = peaks()
     attn_t = statistics.median(attn_ms) * 1e-3
     int8_peak = (pk["bf16_sus"]) * 2.0          # int8 dense = 2x bf16 dense (nominal ratio)
