@@ -22,23 +22,25 @@
 //     never needs rescaling;
 //   * a staging pre-pass turns the key sign bits into +-1 tensor-core
 //     operands once per call (kind::i8 bytes, or e4m3 +-1 for kind::f8f6f4),
-//     laid out tile by tile in the shared-memory order the QK product reads,
-//     each 64-key tile followed by its key scales; for a 2-D relative-position
-//     bias it also writes every table row reversed, in four copies shifted
-//     by one entry, so any bias window a step needs is one aligned copy;
+//     laid out step by step in the shared-memory order the QK product reads,
+//     each 128-key tile followed by its key scales; for a 2-D relative-
+//     position bias it also writes every table row reversed, in four copies
+//     shifted by one entry, so any bias window a step needs is four aligned
+//     copies;
 //   * one loader thread moves everything with bulk copies and TMA (key tiles,
 //     bias windows or dense bias boxes, V tiles) into a 2..4-stage ring: the
 //     loader issues no loads or stores of its own;
 //   * QK runs on tcgen05.mma into three S buffers in TMEM, issued up to two
 //     steps ahead of the softmax; both kinds are exact;
 //   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (each
-//     softmax thread writes its codes over the S columns it has already
-//     read) and s8 V tiles,
-//     accumulating in TMEM across all key tiles;
-//   * the softmax pulls its 64 keys of an S tile out of TMEM with one load and does
-//     its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with a 3-input
-//     max; a bias window is read as reversed copies, four keys per 16-byte
-//     load.
+//     softmax thread writes its codes over the S columns it has already read)
+//     and s8 V tiles, accumulating in TMEM across all key tiles;
+//   * the softmax pulls its 64 keys of an S tile out of TMEM with one load
+//     and does its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with
+//     a 3-input max; a bias window is read as reversed copies, four keys per
+//     16-byte load;
+//   * ring slots and mbarrier parities are counters advanced once per step
+//     (no division by the runtime stage count).
 // Warps 0-7 run the softmax (warp w: TMEM lanes 32 (w % 4) .., keys
 // 64 (w / 4) .. of each step), warp 8 loads, warp 9 issues the MMAs and owns
 // TMEM.

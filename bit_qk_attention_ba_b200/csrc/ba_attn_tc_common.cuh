@@ -1,7 +1,7 @@
 // ba_attn_tc_common.cuh -- pieces shared by the two tensor-core attention
 // kernels (ba_attn_tc.cu: 128-key steps, one row block per CTA;
-// ba_attn_tc_pair.cu: 64-key steps, the same rows of two batch elements per
-// CTA, for a dense bias shared over the batch).
+// ba_attn_tc_pair.cu: 64-key steps, persistent CTAs whose work tiles are the
+// same rows of two batch elements, for a dense bias shared over the batch).
 //
 // Method source: the paper-notes page "BinaryAttention: One-Bit QK-Attention
 // for Vision and Diffusion Transformers" (CVPR 2026), Key designs 1-3.
