@@ -42,10 +42,13 @@ CSRC = os.path.join(ROOT, "bit_qk_attention_ba_b200", "csrc")
 
 def attn_kernel(w, variant):
     """The fused attention kernel a workload runs, and its source file: the
-    CUDA-core kernel for the popcount variant; for a dense bias shared over a
-    batch of two or more, the paired tensor-core kernel; else the 128-key one."""
+    CUDA-core kernel for the popcount variant, the warp-MMA kernel for the .b1
+    variant; otherwise, for a dense bias shared over a batch of two or more,
+    the paired tensor-core kernel, else the 128-key one."""
     if variant == 1:
         return "attn_simt_kernel", os.path.join(CSRC, "ba_attn_simt.cu")
+    if variant == 2:
+        return "attn_b1_kernel", os.path.join(CSRC, "ba_attn_b1.cu")
     if w.bias == "dense" and w.B >= 2:
         return "attn_pair_kernel", os.path.join(CSRC, "ba_attn_tc_pair.cu")
     return "attn_tc_kernel", os.path.join(CSRC, "ba_attn_tc.cu")
@@ -315,7 +318,7 @@ def run_ours(args, w, rank, local_rank, world):
     ops = w.ops
     # pack Q, pack K, V abs-max / quantise / scale, then either the CUDA-core
     # attention or the key staging (+ rel-pos table staging) and the tensor-core one
-    tc_path = ws is not None and args.variant != NAT.BA_QK_POPC
+    tc_path = ws is not None and args.variant not in (NAT.BA_QK_POPC, NAT.BA_QK_MMA_B1)
     fast_rp = kind == NAT.BA_BIAS_RELPOS2D and grid and grid[1] % 128 == 0
     launches_per_step = 5 + (1 + (1 if fast_rp else 0) if tc_path else 0) + 1
     value = aggregate_tops(world, ops, ms)
@@ -430,7 +433,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="hires16k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 3 tcgen05 i8, 4 tcgen05 f8")
+    ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 2 mma.sync b1, 3 tcgen05 i8, 4 tcgen05 f8")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -123,7 +123,8 @@ def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NO
         out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=muq.device)
     kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
     if workspace is None:
-        workspace = attention_workspace(B, H, Nn, d, kind, (gh, gw), device=muq.device)
+        if int(variant) not in (N.BA_QK_POPC, N.BA_QK_MMA_B1):   # the warp-level kernels stage nothing
+            workspace = attention_workspace(B, H, Nn, d, kind, (gh, gw), device=muq.device)
     else:
         _need_cuda(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

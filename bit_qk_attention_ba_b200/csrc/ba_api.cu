@@ -20,6 +20,10 @@ cudaError_t launch_attn_simt(const uint32_t* bq, const float* muq, const uint32_
                              const int8_t* vq, const float* sv, int bias_kind, const float* bias,
                              int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
                              void* out, ba_dtype out_dt, cudaStream_t st);
+cudaError_t launch_attn_b1(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv, int bias_kind, const float* bias,
+                           int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                           void* out, ba_dtype out_dt, cudaStream_t st);
 // Returns cudaErrorNotSupported when the tensor-core path cannot take the shape.
 cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
                            const int8_t* vq, const float* sv, int bias_kind, const float* bias,
@@ -167,9 +171,13 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
         !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)))
         return BA_ERR_INVALID_ARG;
     if (!bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N)) return BA_ERR_INVALID_ARG;
-    if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_TC_I8 && variant != BA_QK_TC_F8)
+    if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_MMA_B1 && variant != BA_QK_TC_I8 &&
+        variant != BA_QK_TC_F8)
         return BA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (variant == BA_QK_MMA_B1)
+        return from_cuda(launch_attn_b1(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
+                                        grid_w, B, H, N, d, out, out_dt, st));
     if (variant == BA_QK_POPC)
         return from_cuda(launch_attn_simt(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
                                           grid_w, B, H, N, d, out, out_dt, st));

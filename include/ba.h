@@ -58,6 +58,7 @@ typedef enum {
 typedef enum {
     BA_QK_AUTO = 0,        /* the fastest path this build has for the shape (tcgen05 kind::i8) */
     BA_QK_POPC = 1,        /* CUDA cores: XOR + popcount on 32-bit words */
+    BA_QK_MMA_B1 = 2,      /* warp mma.sync m16n8k128 .b1 XOR-popcount; PV by mma.sync u8 x s8 */
     BA_QK_TC_I8 = 3,       /* tcgen05 kind::i8, +-1 int8 operands, s32 in TMEM */
     BA_QK_TC_F8 = 4        /* tcgen05 kind::f8f6f4, +-1 e4m3 operands, f32 in TMEM */
 } ba_qk_variant;
@@ -138,7 +139,9 @@ ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
                            void* out, ba_dtype out_dt, void* stream);
 
 /* Same computation with an explicit QK contraction path (ba_qk_variant);
- * BA_ERR_UNSUPPORTED if that path cannot serve the shape. */
+ * BA_ERR_UNSUPPORTED if that path cannot serve the shape.  BA_QK_POPC and
+ * BA_QK_MMA_B1 take every valid shape and ignore the workspace (it may be
+ * NULL with workspace_bytes 0); the tcgen05 paths need the workspace. */
 ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    const uint32_t* bk, const float* muk,
                                    const int8_t* vq, const float* sv,

@@ -84,7 +84,8 @@ def test_bad_dtypes_and_bias_rejected(lib):
     assert lib.ba_attention_fwd(*args, 5, FAKE, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     # out dtype and unknown QK variant
     assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 9, None) == 1
-    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, 2, None) == 1
+    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, 5, None) == 1
+    assert lib.ba_attention_fwd_variant(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, -1, None) == 1
 
 
 def _staged(B, H, N, d, general_relpos=False, keys=128):

@@ -199,7 +199,7 @@ def _small_workload(spec):
 
 
 @pytest.mark.parametrize("spec", SMALL, ids=[s[0] for s in SMALL])
-@pytest.mark.parametrize("variant", [NAT.BA_QK_AUTO, NAT.BA_QK_POPC] + TC_VARIANTS)
+@pytest.mark.parametrize("variant", [NAT.BA_QK_AUTO, NAT.BA_QK_POPC, NAT.BA_QK_MMA_B1] + TC_VARIANTS)
 def test_attention_small_cases(spec, variant):
     w = _small_workload(spec)
     inp = make_inputs(w)
@@ -234,14 +234,16 @@ def test_dominant_bias_selects_value_on_gpu():
     _assert_close(g["out"].cpu().numpy(), ref["out"], inp["v"])
 
 
+@pytest.mark.parametrize("variant", [NAT.BA_QK_AUTO, NAT.BA_QK_MMA_B1])
 @pytest.mark.parametrize("name", list(WORKLOADS))
-def test_attention_full_size(name):
+def test_attention_full_size(name, variant):
     """Every workload at its full size, in the launch configuration the
-    benchmark times.  Small heads are compared in full; for the large ones the
-    oracle computes sampled rows one by one."""
+    benchmark times (the default QK path, and the warp-MMA .b1 one).  Small
+    heads are compared in full; for the large ones the oracle computes sampled
+    rows one by one."""
     w = WORKLOADS[name]
     inp = make_inputs(w)
-    g = _run_gpu(w, inp)
+    g = _run_gpu(w, inp, variant)
     out = g["out"].cpu().numpy()
     del g
     torch.cuda.empty_cache()
