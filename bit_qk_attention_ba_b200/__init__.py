@@ -82,6 +82,35 @@ def quant_v(v, vq=None, sv=None):
     return vq, sv
 
 
+def prepass_qkv(q, k, v, outs=None):
+    """Pack Q and K and quantise V in one call (ba_prepass_qkv): returns
+    (bq, muq, bk, muk, vq, sv), the outputs of pack_qk(q), pack_qk(k) and
+    quant_v(v).  `outs` reuses a previous call's tuple."""
+    torch = _torch()
+    _need_cuda(q, k, v)
+    B, H, Nn, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    if outs is None:
+        dev = q.device
+        outs = (torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=dev),
+                torch.empty((B, H, Nn), dtype=torch.float32, device=dev),
+                torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=dev),
+                torch.empty((B, H, Nn), dtype=torch.float32, device=dev),
+                torch.empty((B, H, d, vq_ld(Nn)), dtype=torch.int8, device=dev),
+                torch.empty((B, H, d), dtype=torch.float32, device=dev))
+    bq, muq, bk, muk, vq, sv = outs
+    N.call("ba_prepass_qkv", _p(q), _p(k), _p(v), _dt(q), B, H, Nn, d, _p(bq), _p(muq), _p(bk), _p(muk),
+           _p(vq), _p(sv), _stream(q.device))
+    return outs
+
+
+def prepass_launches(n, d, dtype):
+    """Kernel launches prepass_qkv makes for this shape (1 when fused)."""
+    torch = _torch()
+    return int(N.lib().ba_prepass_launches(int(n), int(d), N.BA_BF16 if dtype == torch.bfloat16 else N.BA_F32))
+
+
 def _bias_args(bias, bias_kind, ld, grid):
     if bias is None or bias_kind == N.BA_BIAS_NONE:
         return N.BA_BIAS_NONE, None, 0, 0, 0
@@ -161,11 +190,10 @@ def scores_debug(bq, bk, d, z=None):
 
 def forward(q, k, v, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None, out_dtype=None,
             variant=N.BA_QK_AUTO, workspace=None):
-    """The whole hot path: pack Q, pack K, quantise V, fused attention."""
+    """The whole hot path: pack Q, pack K and quantise V (one fused pre-pass
+    call), then the fused attention."""
     d = q.shape[-1]
-    bq, muq = pack_qk(q)
-    bk, muk = pack_qk(k)
-    vq, sv = quant_v(v)
+    bq, muq, bk, muk, vq, sv = prepass_qkv(q, k, v)
     return attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=bias, bias_kind=bias_kind, ld=ld, grid=grid,
                          out_dtype=out_dtype or q.dtype, variant=variant, workspace=workspace)
 

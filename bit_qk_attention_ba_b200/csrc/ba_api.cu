@@ -14,6 +14,10 @@ cudaError_t launch_pack(const void* x, ba_dtype dt, int64_t tokens, int d, uint3
                         float* mu, cudaStream_t st, int sm_count);
 cudaError_t launch_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int8_t* vq,
                            float* sv, cudaStream_t st);
+cudaError_t launch_prepass(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H, int N,
+                           int d, uint32_t* bq, float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv,
+                           cudaStream_t st, int sm_count);
+int prepass_launch_count(int N, int d, ba_dtype dt);
 cudaError_t launch_scores(const uint32_t* bq, const uint32_t* bk, int B, int H, int N, int d,
                           int32_t* z, cudaStream_t st);
 cudaError_t launch_attn_simt(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
@@ -137,6 +141,26 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
     if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
     if (!ptr_ok(v, esize(dt)) || !ptr_ok(vq, 16) || !ptr_ok(sv, 4)) return BA_ERR_INVALID_ARG;
     return from_cuda(launch_quant_v(v, dt, B, H, N, d, vq, sv, static_cast<cudaStream_t>(stream)));
+}
+
+ba_status ba_prepass_qkv(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H, int N, int d,
+                         uint32_t* bq, float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv, void* stream)
+{
+    if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(q, esize(dt)) || !ptr_ok(k, esize(dt)) || !ptr_ok(v, esize(dt))) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
+        !ptr_ok(sv, 4))
+        return BA_ERR_INVALID_ARG;
+    const int sms = sm_count();
+    if (sms <= 0) return BA_ERR_CUDA;
+    return from_cuda(launch_prepass(q, k, v, dt, B, H, N, d, bq, muq, bk, muk, vq, sv,
+                                    static_cast<cudaStream_t>(stream), sms));
+}
+
+int ba_prepass_launches(int N, int d, ba_dtype dt)
+{
+    if (!sizes_ok(1, 1, N, d) || (dt != BA_F32 && dt != BA_BF16)) return -1;
+    return prepass_launch_count(N, d, dt);
 }
 
 ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, int N, int d,

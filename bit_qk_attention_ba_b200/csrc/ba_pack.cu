@@ -5,7 +5,7 @@
 // HBM-bound (read d values, write d/8 bytes + 4 bytes per token), so it is
 // written for coalescing: each lane loads one 16-byte vector, a token is a
 // run of consecutive lanes, and a warp load covers whole tokens back to back.
-#include "ba_common.cuh"
+#include "ba_prepass.cuh"
 
 namespace ba {
 
@@ -76,32 +76,10 @@ __global__ void __launch_bounds__(256)
 pack_row_kernel(const T* __restrict__ x, int64_t tokens, int d, uint32_t* __restrict__ bits,
                 float* __restrict__ mu)
 {
-    constexpr int E = 16 / sizeof(T);
-    constexpr int W = (NV * E + 31) / 32;
+    constexpr int W = (NV * (16 / (int)sizeof(T)) + 31) / 32;
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= tokens) return;
-    const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
-    uint4 raw[NV];
-#pragma unroll
-    for (int k = 0; k < NV; ++k) raw[k] = __ldg(src + k);
-    uint32_t w[W];
-#pragma unroll
-    for (int i = 0; i < W; ++i) w[i] = 0u;
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < NV; ++k) {
-        const T* v = reinterpret_cast<const T*>(&raw[k]);
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int c = k * E + e;
-            const float f = to_f32<T>(v[e]);
-            w[c >> 5] |= (f >= 0.f ? 1u : 0u) << (c & 31);
-            s += fabsf(f);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < W; ++i) bits[t * W + i] = w[i];
-    mu[t] = __fdiv_rn(s, (float)d);
+    pack_token<T, NV>(x + t * d, d, bits + t * W, mu + t);
 }
 
 // General fallback: one warp per token, channel c on lane c % 32.

@@ -6,18 +6,18 @@
 // division), code = round-half-even(v / scale) (IEEE fp32 division), clamped
 // to +-127.
 //
-// When all N keys of one (batch, head) fit in shared memory (the ViT / DiT
-// shapes), one launch does everything with one read of V: one CTA per (b, h)
-// stages the [N, d] block, takes the channel absmax, writes the scales and
-// the codes channel-major.  Otherwise three launches, no scratch memory: (1)
+// When the codes of one (batch, head) fit in shared memory (the ViT / DiT
+// shapes), one launch does everything with one HBM read of V: one CTA per
+// (b, h) takes the channel absmax in a first sweep over the rows, writes the
+// scales, and quantises in a second sweep (served from L2) into channel-major
+// code rows.  Otherwise three launches, no scratch memory: (1)
 // column absmax folded into the sv output with atomicMax on the
 // (non-negative) float bit patterns, (2) quantise a tile of keys and write it
 // transposed into the channel-major [B, H, d, ldv] code layout, (3) turn the
 // stored absmax into the scale.  In both, codes are transposed through
 // shared memory rows whose stride is an odd number of 4-byte words, so the
 // byte writes of a warp (consecutive channels) land in distinct banks.
-#include "ba_common.cuh"
-#include "ba_sm100.cuh"
+#include "ba_prepass.cuh"
 
 namespace ba {
 
@@ -58,31 +58,6 @@ vabsmax_kernel(const T* __restrict__ v, int N, int d, int rows_per_cta, unsigned
         if (red[c]) atomicMax(&amax[bh * d + c], red[c]);
 }
 
-// code = clamp(round_half_even(fl32(x / s)), -127, 127); 0 for an all-zero channel.
-// rs = fl32(1 / s).  Here |x| <= 127 s, so t = fl32(x * rs) is within 3e-5 of
-// x / s and fl32(x / s) within 8e-6 of it: when t is more than 1e-4 away from
-// a rounding boundary (k + 1/2), both round to the same integer, and the code
-// is rint(t); otherwise the IEEE quotient is formed and rounded.  Either way
-// the result equals rounding fl32(x / s).
-__device__ __forceinline__ uint32_t vcode(float x, float s, float rs)
-{
-    if (s == 0.f) return 0u;
-    const float t = x * rs;
-    const float k = (t + 12582912.f) - 12582912.f;     // round-half-even of t (|t| < 2^22)
-    int q;
-    if (0.5f - fabsf(t - k) > 1e-4f) q = (int)k;
-    else q = __float2int_rn(__fdiv_rn(x, s));
-    q = max(-127, min(127, q));
-    return (uint32_t)(q & 0xFF);
-}
-
-// 16 codes of channel row `row` (4-byte aligned, in shared memory) -> 16 bytes of vq.
-__device__ __forceinline__ void store_codes16(int8_t* dst, const uint8_t* row)
-{
-    const uint32_t* q4 = reinterpret_cast<const uint32_t*>(row);
-    *reinterpret_cast<uint4*>(dst) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
-}
-
 // Tile of 64 keys of one (b, h): quantise and store channel-major.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -117,107 +92,16 @@ vquant_kernel(const T* __restrict__ v, int N, int d, int64_t ldv,
     }
 }
 
-// All N keys of one (b, h) in shared memory (tile [N][d] of V, then the codes
-// [d][ldv + 4]): absmax, scale and codes from a single read of V.
+// One CTA per (b, h): absmax, scales and codes with V read from HBM once.
 template <typename T>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(256, 4)
 vquant_small_kernel(const T* __restrict__ v, int N, int d, int64_t ldv, int8_t* __restrict__ vq,
-                    float* __restrict__ sv, unsigned* __restrict__ status)
+                    float* __restrict__ sv)
 {
-    extern __shared__ __align__(16) uint8_t sm_raw[];
-    __shared__ unsigned amax[128];
-    __shared__ float scale[128], rscale[128];
-    T* tile = reinterpret_cast<T*>(sm_raw);
-    const int64_t tile_bytes = (int64_t)N * d * sizeof(T);
-    const int qs = (int)ldv + 4;        // odd number of 4-byte words (ldv % 16 == 0)
-    uint8_t* qt = sm_raw + tile_bytes;
-    __shared__ __align__(8) uint64_t bar;
+    extern __shared__ __align__(16) uint8_t qt[];
+    __shared__ VBlockShared sh;
     const int64_t bh = blockIdx.x;
-    const int tid = threadIdx.x, nt = blockDim.x;
-    // The whole block comes in with bulk copies (at most 64 KB each) on one
-    // mbarrier; the wait is bounded and a timeout only leaves the codes of this
-    // block unwritten after flagging the device status word.
-    if (tid == 0) {
-        sm100::mbar_init(&bar, 1);
-        sm100::fence_mbar_init();
-    }
-    for (int c = tid; c < d; c += nt) amax[c] = 0u;
-    __syncthreads();
-    if (tid == 0) {
-        sm100::mbar_arrive_expect_tx(&bar, (uint32_t)tile_bytes);
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(v + bh * N * d);
-        for (int64_t off = 0; off < tile_bytes; off += 65536) {
-            const uint32_t n = (uint32_t)min((int64_t)65536, tile_bytes - off);
-            sm100::bulk_load(sm_raw + off, src + off, n, &bar);
-        }
-    }
-    const bool landed = sm100::mbar_wait(&bar, 0, nullptr);
-    if (!__syncthreads_and(landed)) {
-        if (tid == 0) atomicOr(status, kStatusTimeoutProducer);
-        return;
-    }
-    // Each thread owns four consecutive channels (d % 4 == 0 here) and walks
-    // the rows: one 8- or 16-byte shared-memory read per row, the scales in
-    // registers.
-    const int G4 = d / 4;
-    const int dr = nt / G4;
-    const bool active = tid < dr * G4;
-    const int c4 = tid % G4, r0 = tid / G4;
-    auto load4 = [&](int r, float (&x)[4]) {
-        if constexpr (sizeof(T) == 2) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(tile + r * d + 4 * c4);
-            const T* h = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) x[e] = to_f32<T>(h[e]);
-        } else {
-            const float4 raw = *reinterpret_cast<const float4*>(tile + r * d + 4 * c4);
-            x[0] = raw.x; x[1] = raw.y; x[2] = raw.z; x[3] = raw.w;
-        }
-    };
-    if (active) {
-        float m[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int r = r0; r < N; r += dr) {
-            float x[4];
-            load4(r, x);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) atomicMax(&amax[4 * c4 + e], __float_as_uint(m[e]));
-    }
-    __syncthreads();
-    for (int c = tid; c < d; c += nt) {
-        const float s = __fdiv_rn(__uint_as_float(amax[c]), 127.0f);
-        scale[c] = s;
-        rscale[c] = __frcp_rn(s);
-        sv[bh * d + c] = s;
-    }
-    __syncthreads();
-    if (active) {
-        float sc[4], rs[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sc[e] = scale[4 * c4 + e];
-            rs[e] = rscale[4 * c4 + e];
-        }
-        uint8_t* qrow = qt + (4 * c4) * qs;
-        const int rows = (int)ldv;
-#pragma unroll 2
-        for (int r = r0; r < rows; r += dr) {
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (r < N) load4(r, x);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                qrow[e * qs + r] = (uint8_t)((r < N) ? vcode(x[e], sc[e], rs[e]) : 0u);
-        }
-    }
-    __syncthreads();
-    const int g16 = (int)(ldv / 16);
-    for (int idx = tid; idx < d * g16; idx += nt) {
-        const int c = idx / g16, g = idx - c * g16;
-        store_codes16(vq + (bh * d + c) * ldv + 16 * g, qt + c * qs + 16 * g);
-    }
+    vblock_quant<T>(v + bh * N * d, N, d, ldv, vq + bh * d * ldv, sv + bh * d, qt, sh);
 }
 
 __global__ void vscale_kernel(float* sv, int64_t n)
@@ -234,14 +118,12 @@ static cudaError_t launch_quant_v_t(const void* v, int B, int H, int N, int d, i
     const int64_t BH = (int64_t)B * H;
     const int64_t ldv = round_up64(N, 16);
     // Single pass when one (b, h) block of V and its codes fit in shared memory.
-    const int64_t small_smem = (int64_t)N * d * sizeof(T) + (int64_t)d * (ldv + 4);
-    if ((d * sizeof(T)) % 16 == 0 && aligned(v, 16) && small_smem <= 200 * 1024) {
+    const int64_t small_smem = vblock_smem_bytes(N, d);
+    if ((d * sizeof(T)) % 16 == 0 && aligned(v, 16) && small_smem <= kVBlockMaxSmem) {
         auto k = vquant_small_kernel<T>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)small_smem);
         if (e != cudaSuccess) return e;
-        unsigned* status = device_status_ptr();
-        if (!status) return cudaErrorInvalidDevice;
-        k<<<(unsigned)BH, 512, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv, status);
+        k<<<(unsigned)BH, 256, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv);
         return cudaGetLastError();
     }
     cudaError_t e = cudaMemsetAsync(sv, 0, sizeof(float) * BH * d, st);

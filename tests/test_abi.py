@@ -48,6 +48,22 @@ def test_pure_helpers(lib):
     assert lib.ba_status_string(4) == b"BA_ERR_DEVICE_STATUS"
 
 
+def test_prepass_launch_count(lib):
+    """One fused launch when a (b, h) block of V fits in shared memory and the
+    token is 2, 4, 8, 9, 12 or 16 vectors of 16 bytes; else pack Q, pack K and
+    one (one-block V) or three (tiled V) quantiser launches."""
+    bf16, f32 = 1, 0
+    assert lib.ba_prepass_launches(577, 64, bf16) == 1        # DeiT-B/384
+    assert lib.ba_prepass_launches(197, 64, f32) == 1         # DeiT-T
+    assert lib.ba_prepass_launches(256, 72, bf16) == 1        # DiT-XL/2 (9 vectors)
+    assert lib.ba_prepass_launches(256, 72, f32) == 3         # 18 vectors: not fused, V in one block
+    assert lib.ba_prepass_launches(16384, 64, bf16) == 5      # HiRes: V tiled
+    assert lib.ba_prepass_launches(90, 33, f32) == 5          # d * 4 not a multiple of 16
+    assert lib.ba_prepass_launches(0, 64, bf16) == -1
+    assert lib.ba_prepass_launches(8, 129, bf16) == -1
+    assert lib.ba_prepass_launches(8, 64, 7) == -1
+
+
 FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced (validation fails first)
 MIS = ctypes.c_void_p((1 << 20) + 1)      # misaligned for every element type
 
@@ -58,6 +74,7 @@ def test_bad_sizes_rejected(lib, B, H, N, d):
     assert lib.ba_pack_qk(FAKE, 1, B, H, N, d, FAKE, FAKE, None) == 1
     assert lib.ba_quant_v(FAKE, 1, B, H, N, d, FAKE, FAKE, None) == 1
     assert lib.ba_scores_debug(FAKE, FAKE, B, H, N, d, FAKE, None) == 1
+    assert lib.ba_prepass_qkv(FAKE, FAKE, FAKE, 1, B, H, N, d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert lib.ba_attention_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, 0, 0, 0,
                                 B, H, N, d, None, 0, FAKE, 0, None) == 1
 
@@ -67,6 +84,11 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.ba_pack_qk(MIS, 1, 1, 1, 8, 64, FAKE, FAKE, None) == 1
     assert lib.ba_quant_v(FAKE, 1, 1, 1, 8, 64, MIS, FAKE, None) == 1
     assert lib.ba_scores_debug(FAKE, None, 1, 1, 8, 64, FAKE, None) == 1
+    pp = [FAKE] * 6
+    assert lib.ba_prepass_qkv(FAKE, None, FAKE, 1, 1, 1, 8, 64, *pp, None) == 1
+    assert lib.ba_prepass_qkv(FAKE, FAKE, MIS, 1, 1, 1, 8, 64, *pp, None) == 1
+    assert lib.ba_prepass_qkv(FAKE, FAKE, FAKE, 1, 1, 1, 8, 64, FAKE, FAKE, FAKE, FAKE, MIS, FAKE, None) == 1
+    assert lib.ba_prepass_qkv(FAKE, FAKE, FAKE, 5, 1, 1, 8, 64, *pp, None) == 1
     args = [FAKE] * 6
     assert lib.ba_attention_fwd(*args[:5], None, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, MIS, 0, None) == 1

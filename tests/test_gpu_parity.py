@@ -59,10 +59,9 @@ def _bias_gpu(inp, w):
 
 
 def _run_gpu(w, inp, variant=NAT.BA_QK_AUTO, out_dtype=torch.float32):
+    """The benchmarked hot path: the fused pre-pass, then the attention call."""
     q, k, v = (_gpu(inp[n], w.dtype) for n in ("q", "k", "v"))
-    bq, muq = ba.pack_qk(q)
-    bk, muk = ba.pack_qk(k)
-    vq, sv = ba.quant_v(v)
+    bq, muq, bk, muk, vq, sv = ba.prepass_qkv(q, k, v)
     out = ba.attention_fwd(bq, muq, bk, muk, vq, sv, w.d, bias=_bias_gpu(inp, w),
                            bias_kind=BIAS_KIND[w.bias], ld=inp["ld"], grid=w.grid,
                            out_dtype=out_dtype, variant=variant)
@@ -99,6 +98,58 @@ def test_pack_and_quant_full_size(name):
     np.testing.assert_array_equal(_vq_natural(vq, w.N), ovq)
     assert vq.shape[-1] == ba.vq_ld(w.N)
     assert not vq[..., w.N:].any()
+
+
+def _check_prepass(w, inp):
+    """prepass_qkv against the oracle (bits, codes and scales bit for bit, mu
+    within fp32 summation error) and against the separate passes (all six
+    outputs bit for bit: they run the same device routines)."""
+    BH = w.B * w.H
+    q, k, v = (_gpu(inp[n], w.dtype) for n in ("q", "k", "v"))
+    fused = ba.prepass_qkv(q, k, v)
+    sep = ba.pack_qk(q) + ba.pack_qk(k) + ba.quant_v(v)
+    torch.cuda.synchronize()
+    for a, b in zip(fused, sep):
+        assert torch.equal(a, b)
+    for key, bits, mu in (("q", fused[0], fused[1]), ("k", fused[2], fused[3])):
+        ob, om = O.pack(inp[key].reshape(BH, w.N, w.d))
+        np.testing.assert_array_equal(_bits(bits).reshape(ob.shape), ob)
+        rel = np.abs(mu.cpu().numpy().reshape(om.shape).astype(np.float64) - om) / np.maximum(om, 1e-30)
+        assert rel.max() <= w.d * 2.0 ** -24 + 2.0 ** -23
+    ovq, osv = O.quant_v(inp["v"].reshape(BH, w.N, w.d))
+    np.testing.assert_array_equal(fused[5].cpu().numpy().reshape(osv.shape), osv)
+    np.testing.assert_array_equal(_vq_natural(fused[4], w.N), ovq)
+    assert not fused[4][..., w.N:].any()
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_prepass_fused_full_size(name):
+    w = WORKLOADS[name]
+    _check_prepass(w, make_inputs(w))
+
+
+PREPASS_SHAPES = [
+    # B, H, N, d, dtype: fused shapes (16-byte vectors per token in {2,4,8,9,12,16}) and fallbacks
+    (2, 3, 1, 64, "bf16"), (2, 3, 77, 16, "bf16"), (1, 2, 300, 72, "bf16"), (1, 2, 129, 96, "bf16"),
+    (1, 2, 200, 128, "bf16"), (2, 2, 197, 64, "f32"), (1, 2, 50, 36, "f32"), (1, 2, 65, 48, "f32"),
+    (1, 1, 90, 8, "f32"), (1, 2, 100, 72, "f32"), (1, 2, 90, 33, "f32"), (1, 1, 1500, 64, "bf16"),
+    (1, 2, 2000, 64, "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape", PREPASS_SHAPES, ids=["x".join(map(str, s)) for s in PREPASS_SHAPES])
+def test_prepass_shapes(shape):
+    B, H, N, d, dtype = shape
+    w = Workload("pp", B, H, N, d, dtype=dtype)
+    inp = make_inputs(w)
+    inp["q"][0, 0, 0, :] = 0.0          # sign(0) and sign(-0) read as +1
+    inp["k"][0, 0, 0, :] = -0.0
+    _check_prepass(w, inp)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    es = 2 if dtype == "bf16" else 4
+    nv = d * es // 16 if (d * es) % 16 == 0 else 0
+    fits = d * (ba.vq_ld(N) + 4) <= 100 * 1024      # the code tile of one (b, h) in shared memory
+    assert (ba.prepass_launches(N, d, tdt) == 1) == (nv in (2, 4, 8, 9, 12, 16) and fits)
 
 
 @pytest.mark.parametrize("N", [300, 5000])
