@@ -5,11 +5,14 @@
 // for Vision and Diffusion Transformers" (CVPR 2026), Key design 1 (sign bits
 // and the per-token scale of Q and K) and Key design 3 (channel-wise int8 V).
 // These are the two HBM-bound steps in front of the attention kernel.  One CTA
-// takes one (b, h): it packs the 2N query and key tokens of the head (one
-// thread per token), then quantises the head's V (channel absmax, then codes
-// transposed through shared memory).  The routines are the ones the separate
+// takes one (b, h): its warps pack the head's N query and N key tokens with
+// coalesced loads staged through shared memory, then the CTA quantises the
+// head's V (channel absmax, then codes transposed through shared memory,
+// reusing the same shared memory).  The routines are the ones the separate
 // passes run (ba_prepass.cuh), so the results are bit-identical to
 // ba_pack_qk + ba_pack_qk + ba_quant_v.
+#include <algorithm>
+
 #include "ba_prepass.cuh"
 
 namespace ba {
@@ -32,18 +35,16 @@ prepass_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __rest
                float* __restrict__ muk, int8_t* __restrict__ vq, float* __restrict__ sv)
 {
     constexpr int W = (NV * (16 / (int)sizeof(T)) + 31) / 32;
-    extern __shared__ __align__(16) uint8_t qt[];
+    extern __shared__ __align__(16) uint8_t smem[];
     __shared__ VBlockShared sh;
     const int64_t bh = blockIdx.x;
     const int64_t base = bh * N;
-    // The sign bits and scales of this head's query tokens, then its key
-    // tokens, consecutive threads on consecutive tokens.
-    for (int t = threadIdx.x; t < 2 * N; t += blockDim.x) {
-        const bool is_k = t >= N;
-        const int64_t tok = base + (is_k ? t - N : t);
-        pack_token<T, NV>((is_k ? k : q) + tok * d, d, (is_k ? bk : bq) + tok * W, (is_k ? muk : muq) + tok);
-    }
-    vblock_quant<T>(v + base * d, N, d, ldv, vq + bh * d * ldv, sv + bh * d, qt, sh);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    uint4* wbuf = reinterpret_cast<uint4*>(smem) + warp * pack_buffer_slots<NV>();
+    pack_tokens_warp<T, NV>(q + base * d, N, d, bq + base * W, muq + base, wbuf, warp, nwarps, lane);
+    pack_tokens_warp<T, NV>(k + base * d, N, d, bk + base * W, muk + base, wbuf, warp, nwarps, lane);
+    __syncthreads();                    // the code tile below reuses the token buffers
+    vblock_quant<T>(v + base * d, N, d, ldv, vq + bh * d * ldv, sv + bh * d, smem, sh);
 }
 
 // 16-byte vectors per token when the fused kernel serves head size d, else 0.
@@ -60,7 +61,8 @@ cudaError_t launch_fused(const void* q, const void* k, const void* v, int BH, in
                          float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv, cudaStream_t st)
 {
     auto kern = prepass_kernel<T, NV>;
-    const int64_t smem = vblock_smem_bytes(N, d);
+    const int64_t tokens_smem = (int64_t)(kThreads / 32) * pack_buffer_slots<NV>() * 16;
+    const int64_t smem = std::max(vblock_smem_bytes(N, d), tokens_smem);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)BH, kThreads, (size_t)smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),

@@ -13,19 +13,16 @@
 
 namespace ba {
 
-// One token of NV 16-byte vectors (E = 16 / sizeof(T) channels each, so
-// d = NV E): the vectors are loaded at once, the sign bits and the |x| sum are
-// built in registers in channel order, and mu = sum / d.
+// One token held as NV 16-byte vectors (E = 16 / sizeof(T) channels each, so
+// d = NV E): the sign bits and the |x| sum are built in registers in channel
+// order, and mu = sum / d.  Every packing path ends here, so all of them give
+// the same bits and the same mu.
 template <typename T, int NV>
-__device__ __forceinline__ void pack_token(const T* __restrict__ x, int d, uint32_t* __restrict__ bits,
-                                           float* __restrict__ mu)
+__device__ __forceinline__ void pack_vectors(const uint4 (&raw)[NV], int d, uint32_t* __restrict__ bits,
+                                             float* __restrict__ mu)
 {
     constexpr int E = 16 / sizeof(T);
     constexpr int W = (NV * E + 31) / 32;
-    const uint4* src = reinterpret_cast<const uint4*>(x);
-    uint4 raw[NV];
-#pragma unroll
-    for (int k = 0; k < NV; ++k) raw[k] = __ldg(src + k);
     uint32_t w[W];
 #pragma unroll
     for (int i = 0; i < W; ++i) w[i] = 0u;
@@ -44,6 +41,61 @@ __device__ __forceinline__ void pack_token(const T* __restrict__ x, int d, uint3
 #pragma unroll
     for (int i = 0; i < W; ++i) bits[i] = w[i];
     *mu = __fdiv_rn(s, (float)d);
+}
+
+// One token read straight from global memory (its NV vectors in flight at once).
+template <typename T, int NV>
+__device__ __forceinline__ void pack_token(const T* __restrict__ x, int d, uint32_t* __restrict__ bits,
+                                           float* __restrict__ mu)
+{
+    const uint4* src = reinterpret_cast<const uint4*>(x);
+    uint4 raw[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) raw[k] = __ldg(src + k);
+    pack_vectors<T, NV>(raw, d, bits, mu);
+}
+
+// Tokens a warp packs per round in pack_tokens_warp, and the 16-byte slots of
+// its shared-memory buffer (one padding slot per token).
+template <int NV> __host__ __device__ constexpr int pack_round_tokens() { return NV <= 9 ? 32 : 16; }
+template <int NV> __host__ __device__ constexpr int pack_buffer_slots() { return pack_round_tokens<NV>() * (NV + 1); }
+
+// The N tokens of one head packed by the warps of a CTA with coalesced loads:
+// per round a warp reads the TPR tokens' TPR NV vectors as consecutive 16-byte
+// loads (each warp load covers 512 contiguous bytes), parks them in its
+// buffer `wbuf` (token-major, stride NV + 1 slots: conflict-free per
+// quarter-warp), and lane l then packs token l from there.
+template <typename T, int NV>
+__device__ __forceinline__ void pack_tokens_warp(const T* __restrict__ x, int N, int d, uint32_t* __restrict__ bits,
+                                                 float* __restrict__ mu, uint4* wbuf, int warp, int nwarps, int lane)
+{
+    constexpr int TPR = pack_round_tokens<NV>();
+    constexpr int NVP = NV + 1;
+    constexpr int PER_LANE = TPR * NV / 32;
+    constexpr int W = (NV * (16 / (int)sizeof(T)) + 31) / 32;
+    const uint4* src = reinterpret_cast<const uint4*>(x);
+    for (int t0 = warp * TPR; t0 < N; t0 += nwarps * TPR) {
+        const int nvec = min(TPR, N - t0) * NV;
+        uint4 r[PER_LANE];
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) {
+            const int vi = k * 32 + lane;
+            r[k] = vi < nvec ? __ldg(src + (int64_t)t0 * NV + vi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) {
+            const int vi = k * 32 + lane;
+            wbuf[vi + vi / NV] = r[k];          // token vi / NV, slot vi % NV
+        }
+        __syncwarp();
+        if (lane < TPR && t0 + lane < N) {
+            uint4 raw[NV];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) raw[v] = wbuf[lane * NVP + v];
+            pack_vectors<T, NV>(raw, d, bits + (int64_t)(t0 + lane) * W, mu + t0 + lane);
+        }
+        __syncwarp();
+    }
 }
 
 // code = clamp(round_half_even(fl32(x / s)), -127, 127); 0 for an all-zero channel.
