@@ -24,7 +24,7 @@ _SRC = os.path.join(_HERE, "ba_oracle.c")
 _LIB = os.path.join(_HERE, "libba_oracle.so")
 _lib = None
 
-BIAS_NONE, BIAS_DENSE, BIAS_RELPOS2D = 0, 1, 2
+BIAS_NONE, BIAS_DENSE, BIAS_RELPOS2D, BIAS_RELPOS2D_CLS = 0, 1, 2, 3
 
 
 def build(force: bool = False) -> str:

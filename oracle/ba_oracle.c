@@ -32,6 +32,12 @@
  *   - The bias is shared over the batch.  Dense: b[h][i][j] at row stride ld.
  *     2-D relative position: token i sits at (i / gw, i % gw); the table index
  *     is (ri - rj + gh - 1) * (2 gw - 1) + (ci - cj + gw - 1).
+ *   - 2-D relative position with a class token (N = gh gw + 1): token 0 is the
+ *     class token and token i >= 1 sits at ((i - 1) / gw, (i - 1) % gw).  The
+ *     page names a relative-position bias but no class token; each head's
+ *     table holds the G = (2 gh - 1)(2 gw - 1) grid entries, then three learned
+ *     scalars: entry G for class query -> patch key, G + 1 for patch query ->
+ *     class key, G + 2 for class -> class.
  */
 #include <math.h>
 #include <pthread.h>
@@ -135,6 +141,17 @@ double bao_bias_value(int kind, const float* bias, int64_t ld, int h, int N,
         int64_t per_head = (int64_t)(2 * gh - 1) * (2 * gw - 1);
         int64_t idx = (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1);
         return (double)bias[(int64_t)h * per_head + idx];
+    }
+    if (kind == 3) {
+        int64_t grid = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+        const float* table = bias + (int64_t)h * (grid + 3);
+        if (i == 0 && j == 0) return (double)table[grid + 2];   /* class -> class */
+        if (i == 0) return (double)table[grid];                 /* class query -> patch key */
+        if (j == 0) return (double)table[grid + 1];             /* patch query -> class key */
+        int pi = i - 1, pj = j - 1;
+        int ri = pi / gw, ci = pi % gw, rj = pj / gw, cj = pj % gw;
+        int64_t idx = (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1);
+        return (double)table[idx];
     }
     return 0.0;
 }

@@ -198,6 +198,44 @@ def test_relpos_structure(oracle, gh, gw):
             assert seen[(dr + 1, dc)] == v + 2 * gw - 1
 
 
+def test_golden_relpos_cls_indexing(oracle):
+    """2-D relative position with a class token, hand-worked on a 2x3 grid
+    plus the class token; with T[k] = k every bias value is its own index."""
+    gh, gw = 2, 3
+    table = np.arange((2 * gh - 1) * (2 * gw - 1) + 3, dtype=np.float32)[None]
+    n = 0
+    with open(os.path.join(GOLDEN, "relpos_cls_2x3.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                i, j, idx = (int(t) for t in line.split())
+                assert oracle.bias_value(3, table, 0, 0, gh * gw + 1, gh, gw, i, j) == idx
+                n += 1
+    assert n == 8
+
+
+@pytest.mark.parametrize("gh,gw", [(3, 4), (2, 2), (1, 5), (4, 1)])
+def test_relpos_cls_structure(oracle, gh, gw):
+    """Brute force over every pair of a grid plus a class token: the class row
+    and column are constant and take the three extra entries; the patch block
+    is the plain rel-pos map of the grid (pinned above) shifted by one token;
+    each head reads its own table."""
+    G = (2 * gh - 1) * (2 * gw - 1)
+    N = gh * gw + 1
+    H = 2
+    table = np.arange(H * (G + 3), dtype=np.float32).reshape(H, G + 3)
+    plain = np.arange(G, dtype=np.float32)[None]
+    for h in range(H):
+        base = h * (G + 3)
+        assert oracle.bias_value(3, table, 0, h, N, gh, gw, 0, 0) == base + G + 2
+        for t in range(1, N):
+            assert oracle.bias_value(3, table, 0, h, N, gh, gw, 0, t) == base + G
+            assert oracle.bias_value(3, table, 0, h, N, gh, gw, t, 0) == base + G + 1
+        for i in range(1, N):
+            for j in range(1, N):
+                want = base + oracle.bias_value(2, plain, 0, 0, N - 1, gh, gw, i - 1, j - 1)
+                assert oracle.bias_value(3, table, 0, h, N, gh, gw, i, j) == want
+
+
 def test_dense_bias_indexing(oracle):
     """Dense bias b[h][i][j] at row stride ld; shared over the batch."""
     H, N, ld = 2, 5, 8
@@ -372,3 +410,29 @@ def test_relpos_forward_matches_dense_expansion(oracle):
     a = oracle.forward(q, k, v, 2, table, 0, gh, gw)["out"]
     b = oracle.forward(q, k, v, 1, dense, N)["out"]
     np.testing.assert_array_equal(a, b)
+
+
+def test_relpos_cls_forward_matches_dense_expansion(oracle):
+    """A rel-pos table with class-token entries gives the same forward as the
+    dense bias built from it through the (pinned) index map, and a dominant
+    class -> class entry makes the class query return the class value."""
+    rng = _rng(23)
+    gh, gw, H, d = 3, 3, 2, 32
+    G = (2 * gh - 1) * (2 * gw - 1)
+    N = gh * gw + 1
+    q = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    k = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    v = rng.standard_normal((1, H, N, d)).astype(np.float32)
+    table = (rng.standard_normal((H, G + 3)) * 0.5).astype(np.float32)
+    dense = np.zeros((H, N, N), np.float32)
+    for h in range(H):
+        for i in range(N):
+            for j in range(N):
+                dense[h, i, j] = oracle.bias_value(3, table, 0, h, N, gh, gw, i, j)
+    a = oracle.forward(q, k, v, 3, table, 0, gh, gw)["out"]
+    b = oracle.forward(q, k, v, 1, dense, N)["out"]
+    np.testing.assert_array_equal(a, b)
+    table[:, G + 2] = 100.0
+    res = oracle.forward(q, k, v, 3, table, 0, gh, gw)
+    vq, sv = res["vq"].reshape(H, N, d), res["sv"].reshape(H, d)
+    np.testing.assert_allclose(res["out"][0, :, 0], vq[:, 0].astype(np.float64) * sv, rtol=1e-12, atol=1e-12)
