@@ -75,9 +75,9 @@ def attn_bytes(w, out_bytes):
     b = 2 * BH * N * W * 4 + 2 * BH * N * 4 + BH * N * d + BH * d * 4 + BH * N * d * out_bytes
     if w.bias == "dense":
         b += w.H * N * N * 4
-    elif w.bias == "relpos2d":
+    elif w.bias in ("relpos2d", "relpos2d_cls"):
         gh, gw = w.grid
-        b += w.H * (2 * gh - 1) * (2 * gw - 1) * 4
+        b += w.H * ((2 * gh - 1) * (2 * gw - 1) + (3 if w.bias == "relpos2d_cls" else 0)) * 4
     return b
 
 

@@ -123,7 +123,8 @@ def _bias_args(bias, bias_kind, ld, grid):
 
 def workspace_bytes(B, H, n, d, bias_kind=N.BA_BIAS_NONE, grid=None) -> int:
     """Device scratch bytes the fused forward needs (ba_attention_workspace_bytes)."""
-    gh, gw = grid if (grid and bias_kind == N.BA_BIAS_RELPOS2D) else (0, 0)
+    rel = bias_kind in (N.BA_BIAS_RELPOS2D, N.BA_BIAS_RELPOS2D_CLS)
+    gh, gw = grid if (grid and rel) else (0, 0)
     nb = N.lib().ba_attention_workspace_bytes(B, H, n, d, int(bias_kind), int(gh), int(gw))
     if nb < 0:
         raise ValueError("invalid sizes or bias arguments for the fused forward")

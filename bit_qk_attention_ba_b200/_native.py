@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(HERE, "libba.so")
 
 BA_OK, BA_ERR_INVALID_ARG, BA_ERR_UNSUPPORTED, BA_ERR_CUDA, BA_ERR_DEVICE_STATUS = 0, 1, 2, 3, 4
 BA_F32, BA_BF16 = 0, 1
-BA_BIAS_NONE, BA_BIAS_DENSE, BA_BIAS_RELPOS2D = 0, 1, 2
+BA_BIAS_NONE, BA_BIAS_DENSE, BA_BIAS_RELPOS2D, BA_BIAS_RELPOS2D_CLS = 0, 1, 2, 3
 BA_QK_AUTO, BA_QK_POPC, BA_QK_MMA_B1, BA_QK_TC_I8, BA_QK_TC_F8 = 0, 1, 2, 3, 4
 
 # name -> (restype, argtypes); mirrors include/ba.h

@@ -99,6 +99,8 @@ static bool bias_ok(int kind, const float* bias, int64_t ld, int gh, int gw, int
     if (kind == BA_BIAS_DENSE) return ptr_ok(bias, 16) && ld >= N && ld % 4 == 0;
     if (kind == BA_BIAS_RELPOS2D)
         return ptr_ok(bias, 4) && gh >= 1 && gw >= 1 && (int64_t)gh * gw == N;
+    if (kind == BA_BIAS_RELPOS2D_CLS)
+        return ptr_ok(bias, 4) && gh >= 1 && gw >= 1 && (int64_t)gh * gw + 1 == N;
     return false;
 }
 
@@ -175,8 +177,10 @@ ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, 
 int64_t ba_attention_workspace_bytes(int B, int H, int N, int d, int bias_kind, int grid_h, int grid_w)
 {
     if (!sizes_ok(B, H, N, d)) return -1;
-    if (bias_kind != BA_BIAS_NONE && bias_kind != BA_BIAS_DENSE && bias_kind != BA_BIAS_RELPOS2D) return -1;
+    if (bias_kind < BA_BIAS_NONE || bias_kind > BA_BIAS_RELPOS2D_CLS) return -1;
     if (bias_kind == BA_BIAS_RELPOS2D && (grid_h < 1 || grid_w < 1 || (int64_t)grid_h * grid_w != N)) return -1;
+    if (bias_kind == BA_BIAS_RELPOS2D_CLS && (grid_h < 1 || grid_w < 1 || (int64_t)grid_h * grid_w + 1 != N))
+        return -1;
     return attn_tc_workspace_bytes(B, H, N, d, bias_kind, grid_h, grid_w);
 }
 

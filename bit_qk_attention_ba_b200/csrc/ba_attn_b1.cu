@@ -116,7 +116,9 @@ attn_b1_kernel(const Params p)
     constexpr int NCH = 2 * NCP;     // 8-channel n-tiles of the PV product
     __shared__ __align__(128) uint32_t s_k[STAGES][KT * 4];      // 16-byte slot per key
     __shared__ __align__(16) float s_mk[STAGES][KT];
-    __shared__ __align__(16) int s_ko[STAGES][BIAS == BA_BIAS_RELPOS2D ? KT : 1];
+    constexpr bool RP = BIAS == BA_BIAS_RELPOS2D || BIAS == BA_BIAS_RELPOS2D_CLS;
+    constexpr int CLS = BIAS == BA_BIAS_RELPOS2D_CLS ? 1 : 0;   // token 0 is a class token
+    __shared__ __align__(16) int s_ko[STAGES][RP ? KT : 1];
     __shared__ __align__(128) uint8_t s_v[STAGES][DVP * VROW];
 
     const int N = p.N, d = p.d;
@@ -146,15 +148,28 @@ attn_b1_kernel(const Params p)
     const float* brow1 = nullptr;
     const float* tab = nullptr;
     int rb0 = 0, rb1 = 0;
+    // Class-token rows and the three class entries (query class -> patch key,
+    // patch query -> class key, class -> class); row r1 = r0 + 8 is never 0.
+    const bool cls0 = CLS && r0 == 0;
+    float c2t = 0.f, t2c = 0.f, c2c = 0.f;
     if (BIAS == BA_BIAS_DENSE) {
         brow0 = p.bias + ((int64_t)head * N + (ok0 ? r0 : 0)) * p.bias_ld;
         brow1 = p.bias + ((int64_t)head * N + (ok1 ? r1 : 0)) * p.bias_ld;
-    } else if (BIAS == BA_BIAS_RELPOS2D) {
+    } else if (RP) {
+        // Patch rows gather table[rb - ko] (ko: the key's patch offset); the
+        // class row gathers from the table centre so every index stays in
+        // range, and its values are replaced below.
         const int w2 = 2 * p.gw - 1;
-        tab = p.bias + (int64_t)head * (2 * p.gh - 1) * w2;
-        const int a0 = ok0 ? r0 : 0, a1 = ok1 ? r1 : 0;
+        const int64_t G = (int64_t)(2 * p.gh - 1) * w2;
+        tab = p.bias + (int64_t)head * (G + 3 * CLS);
+        const int a0 = ok0 && !cls0 ? r0 - CLS : 0, a1 = ok1 ? r1 - CLS : 0;
         rb0 = (a0 / p.gw + p.gh - 1) * w2 + (a0 % p.gw + p.gw - 1);
         rb1 = (a1 / p.gw + p.gh - 1) * w2 + (a1 % p.gw + p.gw - 1);
+        if (CLS) {
+            c2t = __ldg(tab + G);
+            t2c = __ldg(tab + G + 1);
+            c2c = __ldg(tab + G + 2);
+        }
     }
 
     const int T = ceil_div(N, KT);
@@ -174,7 +189,10 @@ attn_b1_kernel(const Params p)
             const int k = tid - KT, j = j0 + k;
             const bool v = j < N;
             cp_async4(sm100::smem_addr(&s_mk[st][k]), p.muk + bh * N + (v ? j : 0), v);
-            if (BIAS == BA_BIAS_RELPOS2D) s_ko[st][k] = v ? (j / p.gw) * (2 * p.gw - 1) + j % p.gw : 0;
+            if (RP) {   // the key's patch offset; -1 marks the class key
+                const int pj = j - CLS;
+                s_ko[st][k] = !v ? 0 : (pj < 0 ? -1 : (pj / p.gw) * (2 * p.gw - 1) + pj % p.gw);
+            }
         }
         if (pass_b) {
             const uint32_t vb = sm100::smem_addr(&s_v[st][0]);
@@ -203,13 +221,18 @@ attn_b1_kernel(const Params p)
                     b0[0] = x0.x; b0[1] = x0.y; b0[2] = x0.z; b0[3] = x0.w;
                     b1v[0] = x1.x; b1v[1] = x1.y; b1v[2] = x1.z; b1v[3] = x1.w;
                 }
-            } else if (BIAS == BA_BIAS_RELPOS2D) {
+            } else if (RP) {
                 const int4 ko = *reinterpret_cast<const int4*>(&s_ko[st][kb]);
                 const int kov[4] = {ko.x, ko.y, ko.z, ko.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     b0[e] = __ldg(tab + rb0 - kov[e]);
                     b1v[e] = __ldg(tab + rb1 - kov[e]);
+                    if (CLS) {
+                        const bool key_cls = kov[e] < 0;
+                        b0[e] = key_cls ? (cls0 ? c2c : t2c) : (cls0 ? c2t : b0[e]);
+                        b1v[e] = key_cls ? t2c : b1v[e];
+                    }
                 }
             }
             const int hm0[4] = {z[2 * hh][0], z[2 * hh][1], z[2 * hh + 1][0], z[2 * hh + 1][1]};
@@ -367,6 +390,8 @@ static void launch_bias(const Params& p, int bias_kind, dim3 grid, cudaStream_t 
         attn_b1_kernel<NCP, W, OutT, BA_BIAS_DENSE><<<grid, 32 * WARPS, 0, st>>>(p);
     else if (bias_kind == BA_BIAS_RELPOS2D)
         attn_b1_kernel<NCP, W, OutT, BA_BIAS_RELPOS2D><<<grid, 32 * WARPS, 0, st>>>(p);
+    else if (bias_kind == BA_BIAS_RELPOS2D_CLS)
+        attn_b1_kernel<NCP, W, OutT, BA_BIAS_RELPOS2D_CLS><<<grid, 32 * WARPS, 0, st>>>(p);
     else
         attn_b1_kernel<NCP, W, OutT, BA_BIAS_NONE><<<grid, 32 * WARPS, 0, st>>>(p);
 }

@@ -31,6 +31,15 @@ __device__ __forceinline__ float bias_at(int kind, const float* __restrict__ bia
         const int64_t per_head = (int64_t)(2 * gh - 1) * (2 * gw - 1);
         return __ldg(bias + h * per_head + (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1));
     }
+    if (kind == BA_BIAS_RELPOS2D_CLS) {   // token 0 is the class token; three class entries follow the grid
+        const int64_t grid = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+        const float* t = bias + h * (grid + 3);
+        if (i == 0) return __ldg(t + grid + (j == 0 ? 2 : 0));
+        if (j == 0) return __ldg(t + grid + 1);
+        const int pi = i - 1, pj = j - 1;
+        const int ri = pi / gw, ci = pi - ri * gw, rj = pj / gw, cj = pj - rj * gw;
+        return __ldg(t + (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1));
+    }
     return 0.f;
 }
 

@@ -155,8 +155,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     const int bh = blockIdx.y;                             // batch * head
     const int h = bh % p.H;
     const int q0 = blockIdx.x * BM;                        // first query row of the CTA
-    const float* tab_h = (BIAS == BA_BIAS_RELPOS2D)
-                             ? p.table + (size_t)h * (2 * p.gh - 1) * (2 * p.gw - 1) : nullptr;
+    // General rel-pos: the head's table (with a class token, the grid entries
+    // are followed by the three class entries, cls3).
+    const size_t rp_grid = (size_t)(2 * p.gh - 1) * (2 * p.gw - 1);
+    const float* tab_h = (BIAS == BA_BIAS_RELPOS2D) ? p.table + h * rp_grid
+                       : (BIAS == BIAS_RP_CLS)      ? p.table + h * (rp_grid + 3) : nullptr;
+    const float* cls3 = (BIAS == BIAS_RP_CLS) ? tab_h + rp_grid : nullptr;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_QREADY], NUM_SOFTMAX_WARPS);
@@ -338,6 +342,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
         const float cq = row_ok ? __ldg(p.muq + (size_t)bh * N + i) * p.q_scale : 0.f;
         const uint64_t cq2 = f2_pack(cq, cq);
         int rel_base = 0, rp_off = 0;
+        bool cls_row = false;
         if (is_relpos(BIAS)) {
             if (BIAS == BIAS_RP_FAST) {
                 // Row r reads window entries 127 - r + k; copy m = (127 - r) % 4
@@ -346,7 +351,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 const int m = sidx & 3;
                 rp_off = m * RP_STRIDE + (sidx - m) + hf * KH;
             } else {
-                const int ri = ie / p.gw, ci = ie - ri * p.gw;
+                // Patch index of the row; the class row (token 0 with a class
+                // token) gathers from the table centre, always in range, and
+                // takes the class entries instead.
+                cls_row = BIAS == BIAS_RP_CLS && ie == 0;
+                const int pe = (BIAS == BIAS_RP_CLS) ? (cls_row ? 0 : ie - 1) : ie;
+                const int ri = pe / p.gw, ci = pe - ri * p.gw;
                 rel_base = (ri + p.gh - 1) * (2 * p.gw - 1) + ci + p.gw - 1;
             }
         }
@@ -383,18 +393,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             if (!pass_b) {
                 if (ragged)
                     softmax_tile<QK, BIAS, false, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
-                                                        nvalid, cq2, neg2, mx, l2, pw);
+                                                        nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 else
                     softmax_tile<QK, BIAS, false, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
-                                                         nvalid, cq2, neg2, mx, l2, pw);
+                                                         nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 mrow = fmax3(mrow, mx[0], mx[1]);
             } else {
                 if (ragged)
                     softmax_tile<QK, BIAS, true, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
-                                                       nvalid, cq2, neg2, mx, l2, pw);
+                                                       nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 else
                     softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
-                                                        nvalid, cq2, neg2, mx, l2, pw);
+                                                        nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 // The u8 codes of these 64 keys go back into this row's lane of
                 // the S buffer, over the first 16 columns of this thread's own
                 // half (already read; the other half's S columns are never
@@ -491,12 +501,14 @@ cudaError_t launch_bias(int kind, const CUtensorMap& tv, const CUtensorMap& tb, 
     if (kind == BA_BIAS_DENSE) return launch_t<QK, OutT, BA_BIAS_DENSE>(tv, tb, p, smem, st);
     if (kind == BIAS_RP_FAST) return launch_t<QK, OutT, BIAS_RP_FAST>(tv, tb, p, smem, st);
     if (kind == BA_BIAS_RELPOS2D) return launch_t<QK, OutT, BA_BIAS_RELPOS2D>(tv, tb, p, smem, st);
+    if (kind == BIAS_RP_CLS) return launch_t<QK, OutT, BIAS_RP_CLS>(tv, tb, p, smem, st);
     return launch_t<QK, OutT, BA_BIAS_NONE>(tv, tb, p, smem, st);
 }
 
 // The kernel variant for an ABI bias kind.
 int kernel_bias(int bias_kind, int gw)
 {
+    if (bias_kind == BA_BIAS_RELPOS2D_CLS) return BIAS_RP_CLS;
     return (bias_kind == BA_BIAS_RELPOS2D && gw % BM == 0) ? BIAS_RP_FAST : bias_kind;
 }
 
@@ -526,12 +538,14 @@ Workspace workspace_layout(int B, int H, int N, int d, int bias_kind, int gh, in
 
 // Staging of the key side, one CTA per (KEYS-key tile, batch*head): +-1 operand
 // bytes in core-matrix order, the key scales (0 past N), and for the general
-// rel-pos bias the key offsets rj (2 gw - 1) + cj.  Keys past N get operand
-// rows of their (zero) sign bits; the kernel masks them out of the softmax.
+// rel-pos bias the key offsets rj (2 gw - 1) + cj of each key's patch (with
+// koff_cls = 1, token 0 is a class token: offset -1, and token j >= 1 is
+// patch j - 1).  Keys past N get operand rows of their (zero) sign bits; the
+// kernel masks them out of the softmax.
 template <int QK, int KEYS>
 __global__ void __launch_bounds__(128)
 stage_k_kernel(const uint32_t* __restrict__ bk, const float* __restrict__ muk, int N, int W, int T,
-               int koff_gw, uint32_t tile, uint8_t* __restrict__ kst)
+               int koff_gw, int koff_cls, uint32_t tile, uint8_t* __restrict__ kst)
 {
     const int t = blockIdx.x;
     const size_t bh = blockIdx.y;
@@ -550,9 +564,9 @@ stage_k_kernel(const uint32_t* __restrict__ bk, const float* __restrict__ muk, i
         const int j = t * KEYS + r;
         mu[r] = (j < N) ? __ldg(muk + bh * N + j) : 0.f;
         if (koff_gw > 0) {
-            const int jj = (j < N) ? j : N - 1;
+            const int jj = ((j < N) ? j : N - 1) - koff_cls;
             const int rj = jj / koff_gw;
-            ko[r] = rj * (2 * koff_gw - 1) + (jj - rj * koff_gw);
+            ko[r] = jj < 0 ? -1 : rj * (2 * koff_gw - 1) + (jj - rj * koff_gw);
         }
     }
 }
@@ -640,7 +654,7 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     p.kst = static_cast<const uint8_t*>(workspace);
     p.rps = (vb == BIAS_RP_FAST) ? reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + ws.rps_off)
                                  : nullptr;
-    p.table = bias_kind == BA_BIAS_RELPOS2D ? bias : nullptr;
+    p.table = (bias_kind == BA_BIAS_RELPOS2D || bias_kind == BA_BIAS_RELPOS2D_CLS) ? bias : nullptr;
     p.out = out;
     p.B = B; p.H = H; p.N = N; p.d = d; p.W = words_for(d); p.dpad = 32 * p.W; p.dv = dv;
     p.n_tiles = ceil_div(N, BN);
@@ -653,15 +667,16 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     {
         const uint32_t tile = (uint32_t)ws.tile;
         uint8_t* kst = static_cast<uint8_t*>(workspace);
-        const int koff_gw = (vb == BA_BIAS_RELPOS2D) ? gw : 0;
+        const int koff_gw = has_koff(vb) ? gw : 0;
+        const int koff_cls = vb == BIAS_RP_CLS ? 1 : 0;
         const int tiles = ceil_div(N, ws.keys);
         dim3 grid(tiles, BH);
         if (ws.keys == 64) {
-            if (f8) stage_k_kernel<QK_F8, 64><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, tile, kst);
-            else stage_k_kernel<QK_I8, 64><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, tile, kst);
+            if (f8) stage_k_kernel<QK_F8, 64><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, koff_cls, tile, kst);
+            else stage_k_kernel<QK_I8, 64><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, koff_cls, tile, kst);
         } else {
-            if (f8) stage_k_kernel<QK_F8, BN><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, tile, kst);
-            else stage_k_kernel<QK_I8, BN><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, tile, kst);
+            if (f8) stage_k_kernel<QK_F8, BN><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, koff_cls, tile, kst);
+            else stage_k_kernel<QK_I8, BN><<<grid, 128, 0, st>>>(bk, muk, N, p.W, tiles, koff_gw, koff_cls, tile, kst);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

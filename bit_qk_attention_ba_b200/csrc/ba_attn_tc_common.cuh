@@ -32,17 +32,25 @@ constexpr int QK_I8 = 0, QK_F8 = 1;
 // grid row and a key tile in one grid row, so its bias is one window of a
 // table row).
 constexpr int BIAS_RP_FAST = 3;
-__host__ __device__ constexpr bool is_relpos(int b) { return b == BA_BIAS_RELPOS2D || b == BIAS_RP_FAST; }
+// The rel-pos bias over a token set whose token 0 is a class token (the ABI's
+// BA_BIAS_RELPOS2D_CLS): the general gather plus the three class entries.
+constexpr int BIAS_RP_CLS = 4;
+__host__ __device__ constexpr bool is_relpos(int b)
+{
+    return b == BA_BIAS_RELPOS2D || b == BIAS_RP_FAST || b == BIAS_RP_CLS;
+}
+// Bias variants whose staged key tiles carry the per-key table offsets.
+__host__ __device__ constexpr bool has_koff(int b) { return b == BA_BIAS_RELPOS2D || b == BIAS_RP_CLS; }
 constexpr size_t kSmemLimit = 227u * 1024u;
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // One staged key tile of `keys` keys: keys x dpad bytes of +-1 operand
-// (K-major core matrices), the key scales, and for the general rel-pos bias
-// the key offsets rj (2 gw - 1) + cj.
+// (K-major core matrices), the key scales, and for the general rel-pos biases
+// the key offsets rj (2 gw - 1) + cj (-1 for a class key).
 __host__ __device__ inline uint32_t tile_bytes(int keys, int dpad, int bias_kind)
 {
-    return (uint32_t)(keys * dpad + keys * 4 + (bias_kind == BA_BIAS_RELPOS2D ? keys * 4 : 0));
+    return (uint32_t)(keys * dpad + keys * 4 + (has_koff(bias_kind) ? keys * 4 : 0));
 }
 
 inline int dv_of(int d) { return (d + 15) / 16 * 16; }
@@ -144,13 +152,21 @@ __device__ __forceinline__ void store_out16(OutT* dst, const uint32_t (&acc)[16]
 // pairs, then either the row maximum (pass A) or P~ = exp(S - m), the row sum
 // and the u8 codes round(255 P~) (pass B).  MASK drops keys >= N.  Two
 // independent max / sum accumulators keep the dependency chains short.
+// For BIAS_RP_CLS, cls3 points at the head's three class entries (class
+// query -> patch key, patch query -> class key, class -> class), a key offset
+// of -1 marks the class key, and cls_row marks the class query's row.
 template <int QK, int BIAS, bool PASS_B, bool MASK>
 __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const float* mks, const uint8_t* bsm_row,
                                              int bsm_sw, const float* rp_copy, const int* koff,
                                              const float* tab_h, int rel_base, int nvalid,
                                              uint64_t cq2, uint64_t neg2, float (&mx)[2], uint64_t (&l2)[2],
-                                             uint32_t (&pw)[16])
+                                             uint32_t (&pw)[16], const float* cls3 = nullptr, bool cls_row = false)
 {
+    float c2t = 0.f, key_cls = 0.f;
+    if (BIAS == BIAS_RP_CLS) {
+        c2t = __ldg(cls3);
+        key_cls = __ldg(cls3 + (cls_row ? 2 : 1));
+    }
     const uint64_t L2E = f2_pack(LOG2E, LOG2E);
     const uint64_t C255 = f2_pack(255.f, 255.f);
     const uint64_t MAGIC = f2_pack(12582912.f, 12582912.f);
@@ -164,10 +180,16 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
             bb = *reinterpret_cast<const float4*>(bsm_row + (k4 >> 3) * 16384 + (((k4 & 7) ^ bsm_sw) << 4));
         } else if (BIAS == BIAS_RP_FAST) {
             bb = *reinterpret_cast<const float4*>(rp_copy + 4 * k4);
-        } else if (BIAS == BA_BIAS_RELPOS2D) {
+        } else if (BIAS == BA_BIAS_RELPOS2D || BIAS == BIAS_RP_CLS) {
             const int4 ko = *reinterpret_cast<const int4*>(koff + 4 * k4);
             bb = make_float4(__ldg(tab_h + rel_base - ko.x), __ldg(tab_h + rel_base - ko.y),
                              __ldg(tab_h + rel_base - ko.z), __ldg(tab_h + rel_base - ko.w));
+            if (BIAS == BIAS_RP_CLS) {
+                bb.x = ko.x < 0 ? key_cls : (cls_row ? c2t : bb.x);
+                bb.y = ko.y < 0 ? key_cls : (cls_row ? c2t : bb.y);
+                bb.z = ko.z < 0 ? key_cls : (cls_row ? c2t : bb.z);
+                bb.w = ko.w < 0 ? key_cls : (cls_row ? c2t : bb.w);
+            }
         }
     };
     float4 mkq[PF], bbq[PF];

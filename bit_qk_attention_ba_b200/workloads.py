@@ -7,7 +7,10 @@ scale, score, softmax or quantisation step lives here.
 The five workloads mirror the model shapes the BinaryAttention paper-notes page
 evaluates (Table 1: DeiT-T/S/B on ImageNet-1K, DeiT-B at 384^2; Table 3:
 DiT-XL/2 at 256^2) plus a 128x128-patch high-resolution ViT, the regime the
-page's motivation section names.  No dataset or trained weight is involved:
+page's motivation section names.  A sixth, deit_b384_rpc, is the DeiT-B at
+384^2 shape with a 2-D relative-position bias over its 24x24 patch grid plus
+the class token, the bias variant Key design 2 names, on a token set with a
+class token.  No dataset or trained weight is involved:
 activations are Gaussian with a per-channel offset, which gives each channel a
 non-zero mean the way trained Q/K/V projections do.
 
@@ -17,8 +20,9 @@ Recipe (all draws from ``numpy.random.default_rng(seed)`` in this order):
     x[b, h, n, c] = offset[h, c] + N(0, 1)
     if outlier_frac > 0: round(outlier_frac * H * d) of the H*d channels,
        drawn without replacement, are multiplied by 8 (after the offset)
-  bias: dense [H, N, N] or a 2-D relative-position table
-        [H, (2 gh - 1) * (2 gw - 1)], entries ~ N(0, bias_std)
+  bias: dense [H, N, N], a 2-D relative-position table
+        [H, (2 gh - 1) * (2 gw - 1)], or that table followed by three class-token
+        entries per head [H, (2 gh - 1) * (2 gw - 1) + 3]; entries ~ N(0, bias_std)
 Values are then rounded to the workload's input dtype (bf16: round to nearest
 even through torch) and returned as float32 numpy arrays holding exactly the
 rounded values.  The dense bias is returned with a padded row stride
@@ -41,8 +45,8 @@ class Workload:
     N: int
     d: int
     dtype: str = "bf16"          # input dtype: "bf16" or "f32"
-    bias: str = "dense"          # "none", "dense" or "relpos2d"
-    grid: tuple = (0, 0)         # (gh, gw) patch grid for "relpos2d"
+    bias: str = "dense"          # "none", "dense", "relpos2d" or "relpos2d_cls"
+    grid: tuple = (0, 0)         # (gh, gw) patch grid for the rel-pos biases
     offset_std: float = 0.5
     outlier_frac: float = 0.0
     bias_std: float = 0.02
@@ -77,6 +81,8 @@ WORKLOADS = {
                         note="DiT-XL/2 at 256^2 latent, 16x16 patches, d=72"),
     "hires16k": Workload("hires16k", 4, 12, 16384, 64, bias="relpos2d", grid=(128, 128),
                          note="high-resolution ViT, 128x128 patch grid, 2-D rel-pos table"),
+    "deit_b384_rpc": Workload("deit_b384_rpc", 32, 12, 577, 64, bias="relpos2d_cls", grid=(24, 24),
+                              note="DeiT-B at 384^2 with a 2-D rel-pos table over 24x24 patches + CLS"),
 }
 
 
@@ -112,10 +118,11 @@ def make_inputs(w: Workload, seed: int | None = None) -> dict:
         padded[:, :, : w.N] = b
         out["bias"] = padded
         out["ld"] = w.ld
-    elif w.bias == "relpos2d":
+    elif w.bias in ("relpos2d", "relpos2d_cls"):
         gh, gw = w.grid
-        assert gh * gw == w.N, "relpos2d needs N == gh * gw"
-        out["bias"] = (rng.standard_normal((w.H, (2 * gh - 1) * (2 * gw - 1)), dtype=np.float32)
+        cls = w.bias == "relpos2d_cls"
+        assert gh * gw + cls == w.N, "rel-pos bias needs N == gh * gw (+ 1 with a class token)"
+        out["bias"] = (rng.standard_normal((w.H, (2 * gh - 1) * (2 * gw - 1) + 3 * cls), dtype=np.float32)
                        * np.float32(w.bias_std))
         out["ld"] = 0
     else:
@@ -124,4 +131,4 @@ def make_inputs(w: Workload, seed: int | None = None) -> dict:
     return out
 
 
-BIAS_KIND = {"none": 0, "dense": 1, "relpos2d": 2}
+BIAS_KIND = {"none": 0, "dense": 1, "relpos2d": 2, "relpos2d_cls": 3}

@@ -51,7 +51,8 @@ typedef enum { BA_F32 = 0, BA_BF16 = 1 } ba_dtype;
 typedef enum {
     BA_BIAS_NONE = 0,
     BA_BIAS_DENSE = 1,     /* fp32 [H, N, ld], b_ij = bias[h][i][j]; ld >= N, ld % 4 == 0 */
-    BA_BIAS_RELPOS2D = 2   /* fp32 [H, (2 gh - 1) * (2 gw - 1)], N == gh * gw, see below */
+    BA_BIAS_RELPOS2D = 2,  /* fp32 [H, (2 gh - 1) * (2 gw - 1)], N == gh * gw, see below */
+    BA_BIAS_RELPOS2D_CLS = 3  /* fp32 [H, (2 gh - 1) * (2 gw - 1) + 3], N == gh * gw + 1, see below */
 } ba_bias_kind;
 
 /* How the binary Q.K contraction runs inside ba_attention_fwd_variant. */
@@ -139,7 +140,14 @@ int64_t ba_attention_workspace_bytes(int B, int H, int N, int d, int bias_kind, 
  *   position.  DENSE: bias_ld is the row stride in floats (>= N, multiple of
  *   4).  RELPOS2D: token i sits at (i / grid_w, i % grid_w), N must equal
  *   grid_h * grid_w, and b_ij = table[h][(ri - rj + grid_h - 1) *
- *   (2 grid_w - 1) + (ci - cj + grid_w - 1)].
+ *   (2 grid_w - 1) + (ci - cj + grid_w - 1)].  RELPOS2D_CLS (a token set with
+ *   a class token; the page names no layout for it, this is the reading
+ *   taken): N must equal grid_h * grid_w + 1, token 0 is the class token and
+ *   token i >= 1 sits at ((i - 1) / grid_w, (i - 1) % grid_w); each head's
+ *   table is the G = (2 grid_h - 1)(2 grid_w - 1) grid entries, indexed as
+ *   for RELPOS2D between patch tokens, then table[h][G] for class query ->
+ *   patch key, table[h][G + 1] for patch query -> class key and
+ *   table[h][G + 2] for class -> class.
  * workspace: device scratch of at least ba_attention_workspace_bytes(...)
  *   bytes, 256-byte aligned (may be NULL when that size is 0); owned by the
  *   caller, used only by work queued on `stream` by this call.  Too small a

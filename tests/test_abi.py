@@ -101,8 +101,13 @@ def test_bad_dtypes_and_bias_rejected(lib):
     assert lib.ba_attention_fwd(*args, 1, FAKE, 4, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     assert lib.ba_attention_fwd(*args, 1, FAKE, 9, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     assert lib.ba_attention_fwd(*args, 1, None, 8, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
-    # rel-pos: N must equal grid_h * grid_w
+    # rel-pos: N must equal grid_h * grid_w (+ 1 with a class token)
     assert lib.ba_attention_fwd(*args, 2, FAKE, 0, 3, 3, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 3, FAKE, 0, 3, 3, 1, 1, 9, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_fwd(*args, 3, None, 0, 3, 3, 1, 1, 10, 64, None, 0, FAKE, 0, None) == 1
+    assert lib.ba_attention_workspace_bytes(1, 1, 9, 64, 3, 3, 3) == -1
+    assert lib.ba_attention_workspace_bytes(1, 1, 10, 64, 3, 3, 3) > 0
+    assert lib.ba_attention_workspace_bytes(1, 1, 10, 64, 4, 3, 3) == -1
     assert lib.ba_attention_fwd(*args, 5, FAKE, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 0, None) == 1
     # out dtype and unknown QK variant
     assert lib.ba_attention_fwd(*args, 0, None, 0, 0, 0, 1, 1, 8, 64, None, 0, FAKE, 9, None) == 1

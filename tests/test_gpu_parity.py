@@ -236,6 +236,10 @@ SMALL = [
     ("d128", 1, 1, 140, 128, "bf16", "none", (0, 0)),
     ("d33", 1, 2, 90, 33, "f32", "dense", (0, 0)),
     ("d1", 1, 1, 40, 1, "f32", "none", (0, 0)),
+    # 2-D rel-pos over a patch grid plus a class token (token 0)
+    ("relpos_cls", 1, 2, 13, 64, "bf16", "relpos2d_cls", (3, 4)),
+    ("relpos_cls_tiles", 2, 3, 301, 64, "bf16", "relpos2d_cls", (15, 20)),
+    ("relpos_cls_d72_f32", 1, 2, 145, 72, "f32", "relpos2d_cls", (12, 12)),
     # dense bias with B >= 2: the paired kernel (two batch elements per CTA)
     ("pair_odd_b", 3, 2, 200, 64, "bf16", "dense", (0, 0)),
     ("pair_d72", 2, 2, 130, 72, "bf16", "dense", (0, 0)),
@@ -281,6 +285,22 @@ def test_dominant_bias_selects_value_on_gpu():
         b[:, i, (5 * i + 1) % w.N] = 100.0
     inp["bias"] = b
     g = _run_gpu(w, inp)
+    ref = _oracle_full(w, inp)
+    _assert_close(g["out"].cpu().numpy(), ref["out"], inp["v"])
+
+
+@pytest.mark.parametrize("variant", [NAT.BA_QK_AUTO, NAT.BA_QK_POPC, NAT.BA_QK_MMA_B1] + TC_VARIANTS)
+def test_relpos_cls_entries_decide_on_gpu(variant):
+    """The three class entries made large (class -> patch +3, patch -> class
+    -4, class -> class +9): the class row and column move far beyond the
+    tolerance if any kernel reads the wrong entry."""
+    w = Workload("cls_dom", 1, 2, 7 * 9 + 1, 64, bias="relpos2d_cls", grid=(7, 9), bias_std=0.3)
+    inp = make_inputs(w)
+    G = 13 * 17
+    inp["bias"][:, G] = 3.0
+    inp["bias"][:, G + 1] = -4.0
+    inp["bias"][:, G + 2] = 9.0
+    g = _run_gpu(w, inp, variant)
     ref = _oracle_full(w, inp)
     _assert_close(g["out"].cpu().numpy(), ref["out"], inp["v"])
 

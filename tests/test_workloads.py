@@ -7,7 +7,11 @@ from bit_qk_attention_ba_b200.workloads import WORKLOADS, make_inputs
 def test_table_matches_the_five_shapes():
     got = {k: (w.B, w.H, w.N, w.d) for k, w in WORKLOADS.items()}
     assert got == {"deit_t": (1, 3, 197, 64), "deit_s": (64, 6, 197, 64), "deit_b384": (32, 12, 577, 64),
-                   "dit_xl2": (32, 16, 256, 72), "hires16k": (4, 12, 16384, 64)}
+                   "dit_xl2": (32, 16, 256, 72), "hires16k": (4, 12, 16384, 64),
+                   "deit_b384_rpc": (32, 12, 577, 64)}
+    w = WORKLOADS["deit_b384_rpc"]
+    assert w.bias == "relpos2d_cls" and w.grid[0] * w.grid[1] + 1 == w.N
+    assert make_inputs(w.scaled(B=1, H=2))["bias"].shape == (2, 47 * 47 + 3)
     assert WORKLOADS["hires16k"].bias == "relpos2d" and WORKLOADS["hires16k"].grid == (128, 128)
     assert WORKLOADS["deit_t"].dtype == "f32"
 
