@@ -70,6 +70,8 @@ def _load():
     lib.bao_attention_fwd_rows.argtypes = [P, P, P, P, P, P, i32, P, i64, i32, i32,
                                            i64, i32, i32, i32, i32, i32, P, i32]
     lib.bao_attention_fwd_rows.restype = i32
+    lib.bao_attention_decode.argtypes = [P, P, P, P, P, P, i32, P, i64, i64, i32, i32, i32, i32, P]
+    lib.bao_attention_decode.restype = None
     _lib = lib
     return lib
 
@@ -187,6 +189,33 @@ def attention_fwd_rows(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, n_
                                           bias_kind, _ptr(b), ld, gh, gw, n_heads, H, N, d, row_lo, row_hi,
                                           _ptr(out), nthreads)
     return out, used
+
+
+def attention_decode(bq, muq, bk, muk, vq, sv, H, d, bias=None, ld=0):
+    """Decode-shaped forward: bq [BH, Nq, W] / muq [BH, Nq] against the cached
+    bk [BH, Nk, W], muk [BH, Nk], vq [BH, Nk, d], sv [BH, d]; optional dense
+    bias [H, Nq, ld].  Returns out [BH, Nq, d] float64."""
+    bq, bk = _c(bq, np.uint32), _c(bk, np.uint32)
+    muq, muk = _c(muq, np.float64), _c(muk, np.float64)
+    vq, sv = _c(vq, np.int8), _c(sv, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    BH, Nq = bq.shape[0], bq.shape[1]
+    Nk = bk.shape[1]
+    out = np.zeros((BH, Nq, d), np.float64)
+    _load().bao_attention_decode(_ptr(bq), _ptr(muq), _ptr(bk), _ptr(muk), _ptr(vq), _ptr(sv),
+                                 1 if b is not None else 0, _ptr(b), int(ld), BH, H, Nq, Nk, d, _ptr(out))
+    return out
+
+
+def decode_forward(q, k, v, bias=None, ld=0):
+    """Whole decode pipeline from raw q [B, H, Nq, d] and the cache's raw
+    k, v [B, H, Nk, d]; returns out [B, H, Nq, d] float64."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    bq, muq = pack(np.asarray(q, np.float32).reshape(B * H, Nq, d))
+    bk, muk = pack(np.asarray(k, np.float32).reshape(B * H, Nk, d))
+    vq, sv = quant_v(np.asarray(v, np.float32).reshape(B * H, Nk, d))
+    return attention_decode(bq, muq, bk, muk, vq, sv, H, d, bias, ld).reshape(B, H, Nq, d)
 
 
 def forward(q, k, v, bias_kind=BIAS_NONE, bias=None, ld=0, gh=0, gw=0, nthreads=0):

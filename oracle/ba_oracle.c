@@ -243,6 +243,56 @@ void bao_attention_rows(const uint32_t* bq, const double* muq,
     free(pq);
 }
 
+/*
+ * Decode-shaped forward: Nq query tokens of each (batch, head) attend to the
+ * Nk cached key / value tokens of the same head (Nq and Nk independent).  The
+ * steps are those of bao_attention_rows:
+ *   S_ij  = muq_i * muk_j * (s_i . t_j) / sqrt(d) + b_ij          (KD2)
+ *   m_i   = max_j S_ij,  P~_ij = exp(S_ij - m_i),  l_i = sum_j P~_ij
+ *   pq_ij = round-half-even(255 * P~_ij)                           (KD3)
+ *   O_ic  = sv_c * sum_j pq_ij * vq_jc / (255 * l_i)               (KD3)
+ * bq [BH, Nq, W], muq [BH, Nq], bk [BH, Nk, W], muk [BH, Nk], vq [BH, Nk, d],
+ * sv [BH, d]; bias kind 0 (none) or 1 (dense: b_ij = bias[h][i][j] at row
+ * stride ld >= Nk, shared over the batch).  out [BH, Nq, d] doubles.
+ */
+void bao_attention_decode(const uint32_t* bq, const double* muq,
+                          const uint32_t* bk, const double* muk,
+                          const int8_t* vq, const float* sv,
+                          int bias_kind, const float* bias, int64_t ld,
+                          int64_t BH, int H, int Nq, int Nk, int d, double* out)
+{
+    const int W = bao_words(d);
+    const double rsd = sqrt((double)d);
+    double* S = (double*)malloc(sizeof(double) * (size_t)Nk);
+    int* pq = (int*)malloc(sizeof(int) * (size_t)Nk);
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % H);
+        for (int i = 0; i < Nq; ++i) {
+            const uint32_t* qi = bq + (bh * Nq + i) * W;
+            for (int j = 0; j < Nk; ++j) {
+                int32_t z = bao_dot_bits(qi, bk + (bh * Nk + j) * W, d);
+                double b = (bias_kind == 1) ? (double)bias[((int64_t)h * Nq + i) * ld + j] : 0.0;
+                S[j] = muq[bh * Nq + i] * muk[bh * Nk + j] * (double)z / rsd + b;
+            }
+            double m = S[0];
+            for (int j = 1; j < Nk; ++j) if (S[j] > m) m = S[j];
+            double l = 0.0;
+            for (int j = 0; j < Nk; ++j) {
+                double p = exp(S[j] - m);
+                l += p;
+                pq[j] = (int)nearbyint(255.0 * p);
+            }
+            for (int c = 0; c < d; ++c) {
+                int64_t acc = 0;
+                for (int j = 0; j < Nk; ++j) acc += (int64_t)pq[j] * vq[(bh * Nk + j) * d + c];
+                out[(bh * Nq + i) * d + c] = (double)sv[bh * d + c] * (double)acc / (255.0 * l);
+            }
+        }
+    }
+    free(S);
+    free(pq);
+}
+
 /* ---- threaded driver over independent (batch, head, row-block) units ---- */
 
 typedef struct {

@@ -436,3 +436,68 @@ def test_relpos_cls_forward_matches_dense_expansion(oracle):
     res = oracle.forward(q, k, v, 3, table, 0, gh, gw)
     vq, sv = res["vq"].reshape(H, N, d), res["sv"].reshape(H, d)
     np.testing.assert_allclose(res["out"][0, :, 0], vq[:, 0].astype(np.float64) * sv, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- decode shape
+
+def _decode_case(seed, B=2, H=3, Nq=4, Nk=53, d=64):
+    rng = _rng(seed)
+    q = (rng.standard_normal((B, H, Nq, d)) + 0.2).astype(np.float32)
+    k = (rng.standard_normal((B, H, Nk, d)) - 0.1).astype(np.float32)
+    v = rng.standard_normal((B, H, Nk, d)).astype(np.float32)
+    return q, k, v
+
+
+def test_decode_rows_match_square_forward(oracle):
+    """Decode of Nq queries against Nk cached keys equals the first Nq rows of
+    the (pinned) square forward over Nk tokens whose first Nq queries are
+    those queries, with the dense bias embedded in the first Nq rows."""
+    q, k, v = _decode_case(29)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    rng = _rng(30)
+    bias = (rng.standard_normal((H, Nq, Nk)) * 0.4).astype(np.float32)
+    q_sq = rng.standard_normal((B, H, Nk, d)).astype(np.float32)
+    q_sq[:, :, :Nq] = q
+    bias_sq = np.zeros((H, Nk, Nk), np.float32)
+    bias_sq[:, :Nq] = bias
+    want = oracle.forward(q_sq, k, v, 1, bias_sq, Nk)["out"][:, :, :Nq]
+    got = oracle.decode_forward(q, k, v, bias, Nk)
+    np.testing.assert_array_equal(got, want)
+    got_nb = oracle.decode_forward(q, k, v)
+    want_nb = oracle.forward(q_sq, k, v)["out"][:, :, :Nq]
+    np.testing.assert_array_equal(got_nb, want_nb)
+
+
+def test_decode_special_cases(oracle):
+    """One cached token returns its dequantised value; a dominant bias entry
+    selects its key; identical keys and no bias give the mean of the
+    dequantised values; permuting the cache leaves the output unchanged."""
+    q, k, v = _decode_case(31, B=1, H=2, Nq=3, Nk=1)
+    out = oracle.decode_forward(q, k, v)
+    vq, sv = oracle.quant_v(v.reshape(2, 1, -1))
+    deq0 = vq[:, 0].astype(np.float64) * sv.astype(np.float64)
+    np.testing.assert_allclose(out.reshape(2, 3, -1), np.broadcast_to(deq0[:, None], (2, 3, 64)),
+                               rtol=1e-13, atol=1e-13)
+
+    q, k, v = _decode_case(32, B=1, H=2, Nq=3, Nk=40)
+    bias = np.zeros((2, 3, 40), np.float32)
+    picks = [7, 0, 39]
+    for i, j in enumerate(picks):
+        bias[:, i, j] = 100.0
+    out = oracle.decode_forward(q, k, v, bias, 40)
+    vq, sv = oracle.quant_v(v.reshape(2, 40, -1))
+    for i, j in enumerate(picks):
+        np.testing.assert_allclose(out[0, :, i], vq[:, j].astype(np.float64) * sv.astype(np.float64),
+                                   rtol=1e-12, atol=1e-12)
+
+    k_same = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    out = oracle.decode_forward(q, k_same, v)
+    vq, sv = oracle.quant_v(v.reshape(2, 40, -1))
+    mean = (vq.astype(np.float64) * sv[:, None].astype(np.float64)).mean(axis=1)
+    np.testing.assert_allclose(out[0], np.broadcast_to(mean[:, None], (2, 3, 64)), rtol=1e-12, atol=1e-12)
+
+    perm = _rng(33).permutation(40)
+    a = oracle.decode_forward(q, k, v, bias, 40)
+    b = oracle.decode_forward(q, k[:, :, perm], v[:, :, perm], bias[:, :, perm].copy(), 40)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
