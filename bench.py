@@ -34,7 +34,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from bit_qk_attention_ba_b200.workloads import BIAS_KIND, WORKLOADS, make_inputs  # noqa: E402
+from bit_qk_attention_ba_b200.workloads import (BIAS_KIND, DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
+                                                make_decode_inputs, make_inputs)
 
 METRIC = "binary attention effective TOPS (4*B*H*N^2*d per step)"
 L2_BYTES = 126 * 2 ** 20
@@ -392,6 +393,151 @@ def run_ours(args, w, rank, local_rank, world):
     return line
 
 
+# ------------------------------------------------------------------ decode shape
+
+def decode_bytes(w, out_bytes):
+    """Algorithmic bytes of one decode call: the cache (key bits, key scales,
+    int8 value codes, value scales), the new queries' bits and scales, and the
+    output."""
+    BH, W = w.B * w.H, (w.d + 31) // 32
+    return BH * w.Nk * (W * 4 + 4 + w.d) + BH * w.d * 4 + BH * w.Nq * (W * 4 + 4) + BH * w.Nq * w.d * out_bytes
+
+
+def run_decode(args, w, rank, local_rank, world):
+    """One step = pack the new queries + the decode forward over the resident
+    cache (packed key bits, key scales, int8 values: built once, as a KV cache
+    is)."""
+    import torch
+    import bit_qk_attention_ba_b200 as ba
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    inp = make_decode_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host_q = torch.from_numpy(inp["q"]).to(tdt).pin_memory()
+    q = host_q.to(dev)
+    bk, muk = ba.pack_qk(torch.from_numpy(inp["k"]).to(tdt).to(dev))
+    vq, sv = ba.quant_v(torch.from_numpy(inp["v"]).to(tdt).to(dev))
+    bq, muq = ba.pack_qk(q)
+    out = torch.empty((w.B, w.H, w.Nq, w.d), dtype=tdt, device=dev)
+    ws = ba.decode_workspace(w.B, w.H, w.Nq, w.Nk, w.d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        ba.pack_qk(q, bq, muq)
+        if i is not None:
+            a0[i].record(stream)
+        ba.attention_decode(bq, muq, bk, muk, vq, sv, w.d, out=out, workspace=ws)
+        if i is not None:
+            a1[i].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(smi_id(dev)) as clk:
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step(i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
+    attn_t = statistics.median(x.elapsed_time(y) for x, y in zip(a0, a1)) * 1e-3
+    status = ba.check_device_status(dev)
+    clocks = clk.summary()
+
+    # end to end: the new queries come from pinned host memory, the output goes back
+    host_out = torch.empty((w.B, w.H, w.Nq, w.d), dtype=tdt).pin_memory()
+    e_steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        qd = host_q.to(dev, non_blocking=True)
+        bqd, muqd = ba.pack_qk(qd)
+        o = ba.attention_decode(bqd, muqd, bk, muk, vq, sv, w.d, out_dtype=tdt, workspace=ws)
+        host_out.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+
+    ms = total_ms / args.steps
+    out_bytes = 2 if tdt == torch.bfloat16 else 4
+    nbytes = decode_bytes(w, out_bytes)
+    pk = peaks()
+    roof = {"bound": "hbm", "achieved": nbytes / attn_t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "kernel": "decode_pv_kernel", "traffic": None, "kernel_us": attn_t * 1e6,
+            "peak_source": "measured HBM copy (%s)" % pk["src"], "algorithmic_bytes": nbytes,
+            "note": "events around ba_attention_decode: three launches (split maxima, codes + PV, combine)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    line = {
+        "metric": METRIC, "value": aggregate_tops(world, w.ops, ms), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8/s8/b1 (QK b1 popcount, PV u8xs8->s32, softmax fp32)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "input_dtype": w.dtype, "bias": "none", "parallelism": "replicas%d" % world,
+                   "l2": "cache larger than L2", "ops": "4*B*H*Nq*Nk*d per step"},
+        "roofline": roof,
+        "e2e": {"value": world * w.ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": host_q.numel() * host_q.element_size(),
+                "d2h_bytes_per_step": host_out.numel() * host_out.element_size(), "ms_per_step": e2e_ms,
+                "cache": "resident on the device"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(w, inp, budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return line
+
+
+def cpu_baseline_decode(w, inp, budget_s=15.0):
+    """The oracle's decode forward on the first heads (packing of the new
+    queries included, the cache packed beforehand), scaled to all heads."""
+    import oracle as O
+    O.build()
+    BH = w.B * w.H
+    q = inp["q"].reshape(BH, w.Nq, w.d)
+    k = inp["k"].reshape(BH, w.Nk, w.d)
+    v = inp["v"].reshape(BH, w.Nk, w.d)
+    heads, t, n = 1, 0.0, 0
+    while True:
+        bk, muk = O.pack(k[n:n + heads])
+        vq, sv = O.quant_v(v[n:n + heads])
+        t0 = time.perf_counter()
+        bq, muq = O.pack(q[n:n + heads])
+        O.attention_decode(bq, muq, bk, muk, vq, sv, w.H, w.d)
+        t += time.perf_counter() - t0
+        n += heads
+        if t >= budget_s or n + heads > BH:
+            break
+        heads = min(heads * 2, BH - n)
+    t_full = t * BH / n
+    return {"value": w.ops / t_full / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d heads (every cached key), %.1f s, scaled to all heads" % (n, BH, t),
+            "seconds_full_workload_est": t_full}
+
+
 # ------------------------------------------------------------------ CPU oracle
 
 def cpu_baseline(w, inp, budget_s=15.0, heads=1):
@@ -454,12 +600,33 @@ def run_reference(args, w, rank, world):
     }
 
 
+def run_reference_decode(args, w, rank, world):
+    if rank != 0:
+        return None
+    inp = make_decode_inputs(w)
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = [cpu_baseline_decode(w, inp, budget_s=per_step) for _ in range(args.warmup + args.steps)][args.warmup:]
+    value = statistics.median(c["value"] for c in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.ops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "input_dtype": w.dtype, "bias": "none", "parallelism": "cpu oracle"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="hires16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="hires16k", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 2 mma.sync b1, 3 tcgen05 i8, 4 tcgen05 f8")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -468,6 +635,15 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, local_rank, world = dist_env()
+    if args.workload in DECODE_WORKLOADS:
+        w = DECODE_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            line = run_reference_decode(args, w, rank, world)
+        else:
+            line = run_decode(args, w, rank, local_rank, world)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+        return
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)

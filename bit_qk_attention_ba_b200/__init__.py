@@ -199,6 +199,37 @@ def forward(q, k, v, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None, out_d
                          out_dtype=out_dtype or q.dtype, variant=variant, workspace=workspace)
 
 
+def attention_decode(bq, muq, bk, muk, vq, sv, d, bias=None, out=None, out_dtype=None, workspace=None):
+    """Decode-shaped forward (ba_attention_decode): bq/muq [B,H,Nq,...] from
+    pack_qk of the queries, bk/muk/vq/sv from pack_qk / quant_v of the cached
+    keys and values; optional dense bias [H, Nq, ld] (ld >= Nk).  Returns out
+    [B,H,Nq,d]; `workspace` (uint8 CUDA tensor) is allocated when not given."""
+    torch = _torch()
+    _need_cuda(bq, muq, bk, muk, vq, sv)
+    B, H, Nq = muq.shape
+    Nk = muk.shape[2]
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=out_dtype or torch.float32, device=muq.device)
+    if workspace is None:
+        workspace = decode_workspace(B, H, Nq, Nk, d, device=muq.device)
+    bp, ld = None, 0
+    if bias is not None:
+        _need_cuda(bias)
+        bp, ld = _p(bias), int(bias.shape[-1])
+    N.call("ba_attention_decode", _p(bq), _p(muq), Nq, _p(bk), _p(muk), _p(vq), _p(sv), Nk, bp, ld, B, H, d,
+           _p(workspace), workspace.numel(), _p(out), _dt(out), _stream(muq.device))
+    return out
+
+
+def decode_workspace(B, H, nq, nk, d, device=None):
+    """A workspace tensor for attention_decode."""
+    torch = _torch()
+    nb = int(N.lib().ba_attention_decode_workspace_bytes(B, H, nq, nk, d))
+    if nb < 0:
+        raise ValueError("invalid decode sizes (1 <= Nq <= 16, d <= 128) or no CUDA device")
+    return torch.empty((max(nb, 256),), dtype=torch.uint8, device=device)
+
+
 def check_device_status(device=None) -> int:
     """Synchronise and return the device status word (0 = no kernel failure)."""
     code = ctypes.c_int(0)

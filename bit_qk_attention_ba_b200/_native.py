@@ -26,6 +26,8 @@ SIGNATURES = {
     "ba_pack_qk": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "ba_quant_v": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "ba_prepass_qkv": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "ba_attention_decode": (_I, [_P, _P, _I, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _P, _I64, _P, _I, _P]),
+    "ba_attention_decode_workspace_bytes": (_I64, [_I, _I, _I, _I, _I]),
     "ba_prepass_launches": (_I, [_I, _I, _I]),
     "ba_attention_workspace_bytes": (_I64, [_I, _I, _I, _I, _I, _I, _I]),
     "ba_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I64,

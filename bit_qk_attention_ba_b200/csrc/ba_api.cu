@@ -35,6 +35,11 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
                            void* workspace, int64_t workspace_bytes,
                            void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st);
 bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d);
+int64_t attn_decode_workspace_bytes(int B, int H, int Nk, int d, int sm_count);
+cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, const uint32_t* bk, const float* muk,
+                               const int8_t* vq, const float* sv, int Nk, const float* bias, int64_t bias_ld,
+                               int B, int H, int d, void* workspace, void* out, ba_dtype out_dt,
+                               cudaStream_t st, int sm_count);
 int64_t attn_tc_workspace_bytes(int B, int H, int N, int d, int bias_kind, int gh, int gw);
 
 // One status word per device; kernels OR failure bits into it.
@@ -236,6 +241,36 @@ ba_status ba_attention_fwd(const uint32_t* bq, const float* muq,
 {
     return ba_attention_fwd_variant(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
                                     B, H, N, d, workspace, workspace_bytes, out, out_dt, BA_QK_AUTO, stream);
+}
+
+static bool decode_sizes_ok(int B, int H, int Nq, int Nk, int d)
+{
+    return Nq >= 1 && Nq <= 16 && sizes_ok(B, H, Nk, d);
+}
+
+int64_t ba_attention_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d)
+{
+    if (!decode_sizes_ok(B, H, Nq, Nk, d)) return -1;
+    const int sms = sm_count();
+    if (sms <= 0) return -1;
+    return attn_decode_workspace_bytes(B, H, Nk, d, sms);
+}
+
+ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
+                              const uint32_t* bk, const float* muk, const int8_t* vq, const float* sv, int Nk,
+                              const float* bias, int64_t bias_ld, int B, int H, int d,
+                              void* workspace, int64_t workspace_bytes, void* out, ba_dtype out_dt, void* stream)
+{
+    if (!decode_sizes_ok(B, H, Nq, Nk, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
+        !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)) || !ptr_ok(workspace, 256))
+        return BA_ERR_INVALID_ARG;
+    if (bias != nullptr && (!ptr_ok(bias, 4) || bias_ld < Nk)) return BA_ERR_INVALID_ARG;
+    const int sms = sm_count();
+    if (sms <= 0) return BA_ERR_CUDA;
+    if (workspace_bytes < attn_decode_workspace_bytes(B, H, Nk, d, sms)) return BA_ERR_INVALID_ARG;
+    return from_cuda(launch_attn_decode(bq, muq, Nq, bk, muk, vq, sv, Nk, bias, bias_ld, B, H, d, workspace, out,
+                                        out_dt, static_cast<cudaStream_t>(stream), sms));
 }
 
 ba_status ba_check_device_status(void* stream, int* code)

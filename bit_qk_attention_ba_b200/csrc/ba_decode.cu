@@ -1,0 +1,351 @@
+// ba_decode.cu -- the BinaryAttention forward in decode shape: Nq (<= 16)
+// query tokens of each (batch, head) attend to an Nk-token cache of packed
+// key sign bits, key scales and int8 value codes.
+//
+// Method source: the paper-notes page "BinaryAttention: One-Bit QK-Attention
+// for Vision and Diffusion Transformers" (CVPR 2026).  Key designs 1-3 define
+// the arithmetic (z = d - 2 popc(q XOR k); S = z mu_q mu_k / sqrt(d) + b;
+// u8 P~ codes against the exact row maximum, int8 V, int32 PV); the page's
+// "Related work and inspiration" section names a compressed KV cache for LLM
+// inference as the place the binary scores carry over to, which is this
+// shape: a 1-bit key cache (d / 8 bytes per key) and an int8 value cache.
+//
+// With few query rows the work is streaming the cache from HBM, so the keys
+// are split over CTAs (split s of a head takes keys [s C, s C + C)), and the
+// exact-maximum reading survives the split: one launch takes each split's row
+// maxima, the next reduces them to the exact maximum m_i, quantises
+// P~ = exp(S - m_i) to u8 codes against it and forms each split's int32 PV
+// sums and P~ row sums; since every split quantises against the same m_i,
+// adding the splits' integer sums is exact.  A last launch adds the splits
+// and applies the epilogue O = sv acc / (255 l).
+#include <math.h>
+
+#include <algorithm>
+
+#include "ba_common.cuh"
+
+namespace ba {
+namespace dec {
+
+constexpr int MAXQ = 16;          // query rows per head this path serves
+constexpr int THREADS = 256;
+constexpr int MAX_CHUNK = 2048;   // keys per split (u8 codes of 16 rows: 32 KB of shared memory)
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct Params {
+    const uint32_t* bq;
+    const float* muq;
+    const uint32_t* bk;
+    const float* muk;
+    const int8_t* vq;
+    const float* sv;
+    const float* bias;   // dense [H, Nq, bias_ld] or null
+    int64_t bias_ld;
+    int H, Nq, Nk, d, S, C;
+    int SA, CA;          // splits of the maximum sweep (wider: its per-key work is small)
+    int64_t ldv;
+    float* pmax;         // [BH][SA][MAXQ] row maxima of the maximum sweep's splits
+    float* psum;         // [BH][S][MAXQ] split sums of P~
+    int* pacc;           // [BH][S][MAXQ][d] int32 PV sums of each split
+    void* out;
+};
+
+__device__ __forceinline__ int dp4a_u8s8(uint32_t a_u8x4, uint32_t b_s8x4, int c)
+{
+    int r;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(a_u8x4), "r"(b_s8x4), "r"(c));
+    return r;
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// The query side of head bh in shared memory: sign words and mu_q / sqrt(d).
+template <int W>
+__device__ __forceinline__ void load_queries(const Params& p, int64_t bh, uint32_t (&qs)[MAXQ][W], float (&cq)[MAXQ])
+{
+    const float rsd = 1.f / sqrtf((float)p.d);
+    for (int e = threadIdx.x; e < p.Nq * W; e += blockDim.x) {
+        const int i = e / W, w = e - i * W;
+        qs[i][w] = __ldg(p.bq + (bh * p.Nq + i) * W + w);
+    }
+    for (int i = threadIdx.x; i < p.Nq; i += blockDim.x) cq[i] = __ldg(p.muq + bh * p.Nq + i) * rsd;
+}
+
+// S_ij for key j of head bh (same expression in both sweeps, so the second
+// sweep reproduces the first's values bit for bit).
+template <int W>
+__device__ __forceinline__ float score(const Params& p, int h, const uint32_t (&kb)[W], float mk,
+                                       const uint32_t (&qs)[MAXQ][W], const float (&cq)[MAXQ], int i, int j)
+{
+    int ham = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) ham += __popc(qs[i][w] ^ kb[w]);
+    const float b = p.bias ? __ldg(p.bias + ((int64_t)h * p.Nq + i) * p.bias_ld + j) : 0.f;
+    return fmaf((float)(p.d - 2 * ham) * mk, cq[i], b);
+}
+
+// Block-wide reduction of MAXQ per-thread values (max or sum), lane order
+// fixed; result in red[i] for every thread after the call.
+template <bool IS_MAX>
+__device__ __forceinline__ void block_reduce(float (&v)[MAXQ], int nq, float (&red)[THREADS / 32][MAXQ],
+                                             float (&out)[MAXQ])
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < MAXQ; ++i) {
+        if (i >= nq) break;
+        float x = v[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float y = __shfl_xor_sync(0xffffffffu, x, o);
+            x = IS_MAX ? fmaxf(x, y) : x + y;
+        }
+        if (lane == 0) red[warp][i] = x;
+    }
+    __syncthreads();
+    if (threadIdx.x < nq) {
+        float x = red[0][threadIdx.x];
+        for (int w = 1; w < THREADS / 32; ++w) x = IS_MAX ? fmaxf(x, red[w][threadIdx.x]) : x + red[w][threadIdx.x];
+        out[threadIdx.x] = x;
+    }
+    __syncthreads();
+}
+
+// Sweep 1: the row maxima of split blockIdx.x of head blockIdx.y.
+template <int W>
+__global__ void __launch_bounds__(THREADS)
+decode_max_kernel(const Params p)
+{
+    __shared__ uint32_t qs[MAXQ][W];
+    __shared__ float cq[MAXQ];
+    __shared__ float red[THREADS / 32][MAXQ];
+    __shared__ float res[MAXQ];
+    const int s = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int h = (int)(bh % p.H);
+    load_queries<W>(p, bh, qs, cq);
+    __syncthreads();
+    float mx[MAXQ];
+#pragma unroll
+    for (int i = 0; i < MAXQ; ++i) mx[i] = -INFINITY;
+    const int j1 = min(p.Nk, (s + 1) * p.CA);
+#pragma unroll 8
+    for (int j = s * p.CA + threadIdx.x; j < j1; j += blockDim.x) {
+        uint32_t kb[W];
+#pragma unroll
+        for (int w = 0; w < W; ++w) kb[w] = __ldg(p.bk + (bh * p.Nk + j) * W + w);
+        const float mk = __ldg(p.muk + bh * p.Nk + j);
+#pragma unroll
+        for (int i = 0; i < MAXQ; ++i) {
+            if (i >= p.Nq) break;
+            mx[i] = fmaxf(mx[i], score<W>(p, h, kb, mk, qs, cq, i, j));
+        }
+    }
+    block_reduce<true>(mx, p.Nq, red, res);
+    if (threadIdx.x < p.Nq) p.pmax[(bh * p.SA + s) * MAXQ + threadIdx.x] = res[threadIdx.x];
+}
+
+// Sweep 2: exact m_i from the split maxima, u8 codes of this split's keys,
+// the split's P~ sums and int32 PV sums.
+template <int W>
+__global__ void __launch_bounds__(THREADS, 3)
+decode_pv_kernel(const Params p)
+{
+    __shared__ uint32_t qs[MAXQ][W];
+    __shared__ float cq[MAXQ];
+    __shared__ float negm[MAXQ];
+    __shared__ float red[THREADS / 32][MAXQ];
+    __shared__ float res[MAXQ];
+    __shared__ __align__(16) uint8_t pq[MAXQ][MAX_CHUNK];
+    __shared__ int sacc[MAXQ][128];
+    const int s = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int h = (int)(bh % p.H);
+    load_queries<W>(p, bh, qs, cq);
+    if (threadIdx.x < p.Nq) {
+        float m = -INFINITY;
+        for (int t = 0; t < p.SA; ++t) m = fmaxf(m, p.pmax[(bh * p.SA + t) * MAXQ + threadIdx.x]);
+        negm[threadIdx.x] = -m * LOG2E;
+    }
+    for (int e = threadIdx.x; e < MAXQ * 128; e += blockDim.x) (&sacc[0][0])[e] = 0;
+    __syncthreads();
+    const int j0 = s * p.C;
+    const int len = min(p.Nk - j0, p.C);
+    const int len16 = (len + 15) & ~15;
+    float l[MAXQ];
+#pragma unroll
+    for (int i = 0; i < MAXQ; ++i) l[i] = 0.f;
+#pragma unroll 4
+    for (int jj = threadIdx.x; jj < len16; jj += blockDim.x) {
+        const int j = j0 + jj;
+        const bool live = jj < len;
+        uint32_t kb[W];
+#pragma unroll
+        for (int w = 0; w < W; ++w) kb[w] = live ? __ldg(p.bk + (bh * p.Nk + j) * W + w) : 0u;
+        const float mk = live ? __ldg(p.muk + bh * p.Nk + j) : 0.f;
+#pragma unroll
+        for (int i = 0; i < MAXQ; ++i) {
+            if (i >= p.Nq) break;
+            uint32_t code = 0u;
+            if (live) {
+                const float pr = ex2(fmaf(score<W>(p, h, kb, mk, qs, cq, i, j), LOG2E, negm[i]));
+                l[i] += pr;
+                code = (uint32_t)__float2int_rn(255.f * pr);
+            }
+            pq[i][jj] = (uint8_t)code;
+        }
+    }
+    block_reduce<false>(l, p.Nq, red, res);   // also orders the code writes before the reads below
+    if (threadIdx.x < p.Nq) p.psum[(bh * p.S + s) * MAXQ + threadIdx.x] = res[threadIdx.x];
+
+    // PV: thread (g, c) takes channel c and key slice g of the split (G =
+    // THREADS / d slices of whole 16-key groups), for every row; 16 keys per
+    // step: one 16-byte load of the channel's codes, one 16-byte read of each
+    // row's P codes (the same address across the warp), four dp4a each.  The
+    // slices' sums meet in shared memory (integer adds: order-free).
+    const int d = p.d;
+    const int G = THREADS / d;
+    const bool pv_thread = threadIdx.x < G * d;
+    const int c = threadIdx.x % d, g = threadIdx.x / d;
+    const int groups = len16 / 16;
+    const int k_lo = pv_thread ? 16 * (groups * g / G) : 0;
+    const int k_hi = pv_thread ? 16 * (groups * (g + 1) / G) : 0;
+    int acc[MAXQ];
+#pragma unroll
+    for (int i = 0; i < MAXQ; ++i) acc[i] = 0;
+    const int8_t* vrow = p.vq + (bh * d + c) * p.ldv + j0;
+    // Eight independent 16-byte loads of the channel's codes in flight per
+    // thread, then the rows' dot products.
+    constexpr int U = 8;
+    for (int k0 = k_lo; k0 < k_hi; k0 += 16 * U) {
+        uint4 vv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            vv[u] = (k0 + 16 * u < k_hi) ? __ldg(reinterpret_cast<const uint4*>(vrow + k0 + 16 * u))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + 16 * u;
+            if (k >= k_hi) break;
+#pragma unroll
+            for (int i = 0; i < MAXQ; ++i) {
+                if (i >= p.Nq) break;
+                const uint4 a = *reinterpret_cast<const uint4*>(&pq[i][k]);
+                int t = acc[i];
+                t = dp4a_u8s8(a.x, vv[u].x, t);
+                t = dp4a_u8s8(a.y, vv[u].y, t);
+                t = dp4a_u8s8(a.z, vv[u].z, t);
+                acc[i] = dp4a_u8s8(a.w, vv[u].w, t);
+            }
+        }
+    }
+    if (pv_thread) {
+#pragma unroll
+        for (int i = 0; i < MAXQ; ++i) {
+            if (i >= p.Nq) break;
+            atomicAdd(&sacc[i][c], acc[i]);
+        }
+    }
+    __syncthreads();
+    int* dst = p.pacc + ((bh * p.S + s) * MAXQ) * d;
+    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) dst[e] = sacc[e / d][e % d];
+}
+
+// The splits added (int64 code sums, P~ sums in split order) and the epilogue.
+template <typename OutT>
+__global__ void __launch_bounds__(THREADS)
+decode_combine_kernel(const Params p)
+{
+    const int64_t bh = blockIdx.x;
+    const int d = p.d;
+    OutT* out = static_cast<OutT*>(p.out);
+    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) {
+        const int i = e / d, c = e - i * d;
+        long long acc = 0;
+        float l = 0.f;
+        for (int s = 0; s < p.S; ++s) {
+            acc += p.pacc[((bh * p.S + s) * MAXQ + i) * d + c];
+            l += p.psum[(bh * p.S + s) * MAXQ + i];
+        }
+        const float o = __ldg(p.sv + bh * d + c) * (float)acc / (255.f * l);
+        if constexpr (sizeof(OutT) == 2) out[(bh * p.Nq + i) * d + c] = __float2bfloat16_rn(o);
+        else out[(bh * p.Nq + i) * d + c] = o;
+    }
+}
+
+// Splits per head: enough CTAs for about four per SM, at most MAX_CHUNK keys
+// and at least 256 keys per split (chunk lengths a multiple of 16).
+struct Split {
+    int S, C;     // PV sweep: splits and keys per split
+    int SA, CA;   // maximum sweep: four PV splits per split
+};
+
+inline Split choose_split(int64_t BH, int Nk, int sm_count)
+{
+    const int64_t want = (4 * (int64_t)sm_count + BH - 1) / BH;
+    int S = (int)std::max<int64_t>(1, std::min<int64_t>(want, (Nk + 255) / 256));
+    S = std::max(S, (Nk + MAX_CHUNK - 1) / MAX_CHUNK);
+    int C = (Nk + S - 1) / S;
+    C = (C + 15) / 16 * 16;
+    S = (Nk + C - 1) / C;
+    const int CA = 4 * C;
+    return {S, C, (Nk + CA - 1) / CA, CA};
+}
+
+inline int64_t workspace_bytes(int64_t BH, int Nk, int d, int sm_count)
+{
+    const Split sp = choose_split(BH, Nk, sm_count);
+    const int64_t rows = BH * sp.S * MAXQ;
+    return rows * 4 * 2 + rows * d * 4;
+}
+
+template <int W>
+cudaError_t launch_w(Params p, int64_t BH, ba_dtype out_dt, cudaStream_t st)
+{
+    decode_max_kernel<W><<<dim3(p.SA, (unsigned)BH), THREADS, 0, st>>>(p);
+    decode_pv_kernel<W><<<dim3(p.S, (unsigned)BH), THREADS, 0, st>>>(p);
+    if (out_dt == BA_BF16)
+        decode_combine_kernel<__nv_bfloat16><<<(unsigned)BH, THREADS, 0, st>>>(p);
+    else
+        decode_combine_kernel<float><<<(unsigned)BH, THREADS, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace dec
+
+int64_t attn_decode_workspace_bytes(int B, int H, int Nk, int d, int sm_count)
+{
+    return dec::workspace_bytes((int64_t)B * H, Nk, d, sm_count);
+}
+
+cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, const uint32_t* bk, const float* muk,
+                               const int8_t* vq, const float* sv, int Nk, const float* bias, int64_t bias_ld,
+                               int B, int H, int d, void* workspace, void* out, ba_dtype out_dt,
+                               cudaStream_t st, int sm_count)
+{
+    const int64_t BH = (int64_t)B * H;
+    const dec::Split sp = dec::choose_split(BH, Nk, sm_count);
+    const int64_t rows = BH * sp.S * dec::MAXQ;
+    dec::Params p;
+    p.bq = bq; p.muq = muq; p.bk = bk; p.muk = muk; p.vq = vq; p.sv = sv;
+    p.bias = bias; p.bias_ld = bias_ld;
+    p.H = H; p.Nq = Nq; p.Nk = Nk; p.d = d; p.S = sp.S; p.C = sp.C; p.SA = sp.SA; p.CA = sp.CA;
+    p.ldv = round_up64(Nk, 16);
+    p.pmax = static_cast<float*>(workspace);
+    p.psum = p.pmax + rows;
+    p.pacc = reinterpret_cast<int*>(p.psum + rows);
+    p.out = out;
+    switch (words_for(d)) {
+        case 1: return dec::launch_w<1>(p, BH, out_dt, st);
+        case 2: return dec::launch_w<2>(p, BH, out_dt, st);
+        case 3: return dec::launch_w<3>(p, BH, out_dt, st);
+        default: return dec::launch_w<4>(p, BH, out_dt, st);
+    }
+}
+
+}  // namespace ba

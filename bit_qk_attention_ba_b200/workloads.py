@@ -132,3 +132,42 @@ def make_inputs(w: Workload, seed: int | None = None) -> dict:
 
 
 BIAS_KIND = {"none": 0, "dense": 1, "relpos2d": 2, "relpos2d_cls": 3}
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq new query tokens per (batch, head) against an Nk-token cache."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    dtype: str = "bf16"
+    offset_std: float = 0.5
+    seed: int = 0
+    note: str = ""
+
+    @property
+    def ops(self) -> float:
+        """Effective operations of one decode call, 4*B*H*Nq*Nk*d."""
+        return 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
+
+
+DECODE_WORKLOADS = {
+    "decode_16k": DecodeWorkload("decode_16k", 32, 12, 1, 16384, 64,
+                                 note="one new query per head against a 16384-token cache, DeiT-B-sized heads"),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: int | None = None) -> dict:
+    """Draw the new queries q [B, H, Nq, d] and the cache's raw keys and
+    values k, v [B, H, Nk, d] (per-channel offsets as in make_inputs)."""
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    out = {}
+    for name, n in (("q", w.Nq), ("k", w.Nk), ("v", w.Nk)):
+        offset = rng.standard_normal((w.H, w.d), dtype=np.float32) * np.float32(w.offset_std)
+        x = rng.standard_normal((w.B, w.H, n, w.d), dtype=np.float32)
+        x += offset[None, :, None, :]
+        out[name] = _round_dtype(x, w.dtype)
+    return out

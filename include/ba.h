@@ -196,6 +196,32 @@ ba_status ba_attention_fwd_noalloc(const uint32_t* bq, const float* muq,
                                    void* out, ba_dtype out_dt, void* stream);
 
 /*
+ * KD1-KD3 in decode shape: Nq query tokens of each (b, h) attend to an
+ * Nk-token cache of the same head (the compressed KV cache the page's
+ * "Related work and inspiration" section points to for LLM inference).
+ *   bq [B, H, Nq, W], muq [B, H, Nq]  : ba_pack_qk of the queries (N = Nq)
+ *   bk [B, H, Nk, W], muk [B, H, Nk]  : ba_pack_qk of the cached keys (N = Nk)
+ *   vq [B, H, d, ba_vq_ld(Nk)], sv [B, H, d] : ba_quant_v of the cached values
+ *   bias : NULL, or dense fp32 [H, Nq, bias_ld] (bias_ld >= Nk), shared over B
+ *   out  : [B, H, Nq, d] in out_dt
+ * 1 <= Nq <= 16.  The same arithmetic as ba_attention_fwd (exact row maximum,
+ * u8 codes of P~ against it, l the sum of the unquantised P~).  The keys are
+ * split over CTAs; every split quantises against the exact maximum, so the
+ * splits' int32 sums add exactly.  workspace: device scratch of at least
+ * ba_attention_decode_workspace_bytes(B, H, Nq, Nk, d) bytes, 256-byte
+ * aligned, owned by the caller, rewritten by every call.  Three kernel
+ * launches on `stream`.
+ */
+ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
+                              const uint32_t* bk, const float* muk, const int8_t* vq, const float* sv, int Nk,
+                              const float* bias, int64_t bias_ld, int B, int H, int d,
+                              void* workspace, int64_t workspace_bytes, void* out, ba_dtype out_dt, void* stream);
+
+/* Workspace bytes ba_attention_decode needs on the current device; -1 for
+ * invalid sizes or when no device is available. */
+int64_t ba_attention_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+
+/*
  * KD1 -- the integer binary score matrix, for checking and debugging.
  *   z : [B, H, N, N] int32, z[b][h][i][j] = d - 2 popcount(bq_i XOR bk_j).
  */

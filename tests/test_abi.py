@@ -124,6 +124,21 @@ def _staged(B, H, N, d, general_relpos=False, keys=128):
     return B * H * ((N + keys - 1) // keys) * tile
 
 
+def test_decode_arguments_checked(lib):
+    """ba_attention_decode rejects bad sizes, pointers and bias strides before
+    touching the device."""
+    p = [FAKE] * 2
+    good = dict(Nq=1, Nk=64, B=1, H=1, d=64)
+    def call(Nq=1, Nk=64, B=1, H=1, d=64, bq=FAKE, vq=FAKE, bias=None, ld=0, ws=FAKE, out_dt=0):
+        return lib.ba_attention_decode(bq, FAKE, Nq, FAKE, FAKE, vq, FAKE, Nk, bias, ld, B, H, d,
+                                       ws, 1 << 30, FAKE, out_dt, None)
+    assert call(Nq=0) == 1 and call(Nq=17) == 1 and call(Nk=0) == 1 and call(d=129) == 1
+    assert call(bq=None) == 1 and call(vq=MIS) == 1 and call(ws=None) == 1 and call(out_dt=5) == 1
+    assert call(bias=FAKE, ld=32) == 1                     # ld < Nk
+    assert lib.ba_attention_decode_workspace_bytes(1, 1, 17, 64, 64) == -1
+    assert lib.ba_attention_decode_workspace_bytes(1, 1, 0, 64, 64) == -1
+
+
 def test_workspace_size_query(lib):
     """Workspace = staged key tiles, and for a rel-pos grid width that is a
     multiple of 128 four shifted copies of every reversed table row."""
