@@ -483,7 +483,9 @@ def run_decode(args, w, rank, local_rank, world):
     nbytes = decode_bytes(w, out_bytes)
     pk = peaks()
     roof = {"bound": "hbm", "achieved": nbytes / attn_t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "kernel": "decode_pv_kernel", "traffic": None, "kernel_us": attn_t * 1e6,
+            "kernel": "decode_pv_kernel",
+            "traffic": recorded_traffic("decode_pv_kernel", os.path.join(CSRC, "ba_decode.cu"), w.name),
+            "kernel_us": attn_t * 1e6,
             "peak_source": "measured HBM copy (%s)" % pk["src"], "algorithmic_bytes": nbytes,
             "note": "events around ba_attention_decode: three launches (split maxima, codes + PV, combine)"}
     roof["frac"] = roof["achieved"] / roof["peak"]

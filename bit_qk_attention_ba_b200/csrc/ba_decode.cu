@@ -43,6 +43,7 @@ struct Params {
     int64_t bias_ld;
     int H, Nq, Nk, d, S, C;
     int SA, CA;          // splits of the maximum sweep (wider: its per-key work is small)
+    int bk_vec;          // key bits 4 W-byte aligned: one vector load per key (W = 2 or 4)
     int64_t ldv;
     float* pmax;         // [BH][SA][MAXQ] row maxima of the maximum sweep's splits
     float* psum;         // [BH][S][MAXQ] split sums of P~
@@ -74,6 +75,29 @@ __device__ __forceinline__ void load_queries(const Params& p, int64_t bh, uint32
         qs[i][w] = __ldg(p.bq + (bh * p.Nq + i) * W + w);
     }
     for (int i = threadIdx.x; i < p.Nq; i += blockDim.x) cq[i] = __ldg(p.muq + bh * p.Nq + i) * rsd;
+}
+
+// The W sign words of key j: one 8- or 16-byte load when the rows are aligned for it.
+template <int W>
+__device__ __forceinline__ void load_key(const Params& p, int64_t bh, int j, uint32_t (&kb)[W])
+{
+    const uint32_t* src = p.bk + (bh * p.Nk + j) * W;
+    if constexpr (W == 2) {
+        if (p.bk_vec) {
+            const uint2 t = __ldg(reinterpret_cast<const uint2*>(src));
+            kb[0] = t.x;
+            kb[1] = t.y;
+            return;
+        }
+    } else if constexpr (W == 4) {
+        if (p.bk_vec) {
+            const uint4 t = __ldg(reinterpret_cast<const uint4*>(src));
+            kb[0] = t.x; kb[1] = t.y; kb[2] = t.z; kb[3] = t.w;
+            return;
+        }
+    }
+#pragma unroll
+    for (int w = 0; w < W; ++w) kb[w] = __ldg(src + w);
 }
 
 // S_ij for key j of head bh (same expression in both sweeps, so the second
@@ -137,8 +161,7 @@ decode_max_kernel(const Params p)
 #pragma unroll 8
     for (int j = s * p.CA + threadIdx.x; j < j1; j += blockDim.x) {
         uint32_t kb[W];
-#pragma unroll
-        for (int w = 0; w < W; ++w) kb[w] = __ldg(p.bk + (bh * p.Nk + j) * W + w);
+        load_key<W>(p, bh, j, kb);
         const float mk = __ldg(p.muk + bh * p.Nk + j);
 #pragma unroll
         for (int i = 0; i < MAXQ; ++i) {
@@ -186,7 +209,8 @@ decode_pv_kernel(const Params p)
         const bool live = jj < len;
         uint32_t kb[W];
 #pragma unroll
-        for (int w = 0; w < W; ++w) kb[w] = live ? __ldg(p.bk + (bh * p.Nk + j) * W + w) : 0u;
+        for (int w = 0; w < W; ++w) kb[w] = 0u;
+        if (live) load_key<W>(p, bh, j, kb);
         const float mk = live ? __ldg(p.muk + bh * p.Nk + j) : 0.f;
 #pragma unroll
         for (int i = 0; i < MAXQ; ++i) {
@@ -335,6 +359,8 @@ cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, con
     p.bq = bq; p.muq = muq; p.bk = bk; p.muk = muk; p.vq = vq; p.sv = sv;
     p.bias = bias; p.bias_ld = bias_ld;
     p.H = H; p.Nq = Nq; p.Nk = Nk; p.d = d; p.S = sp.S; p.C = sp.C; p.SA = sp.SA; p.CA = sp.CA;
+    const int W = words_for(d);
+    p.bk_vec = (W == 2 || W == 4) && aligned(bk, 4u * W);
     p.ldv = round_up64(Nk, 16);
     p.pmax = static_cast<float*>(workspace);
     p.psum = p.pmax + rows;
