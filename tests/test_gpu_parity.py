@@ -2,9 +2,10 @@
 
 Integer outputs (sign bits, int8 V codes, binary scores) must match bit for
 bit.  Floating outputs: mu within fp32 summation error; the attention output
-within max-abs 2e-2 and mean-abs 2e-3 of the oracle (exact row max, fp64) on
-unit-scale V -- errors are divided by max(1, std of the value channel) so the
-x8 outlier channels of the DeiT-S workload get the same relative budget.  The
+within max-abs 2e-2 and mean-abs 2e-3 of the oracle (exact row max, fp64),
+asserted on the raw errors and again on the errors divided by max(1, std of
+the value channel) -- the reading of "on unit-scale V" for the x8 outlier
+channels of the DeiT-S workload, which the raw check already implies.  The
 GPU also takes the exact row maximum (two sweeps over the keys) but computes in
 fp32, so a code sitting on a rounding boundary can move by one unit; that is
 what the tolerance covers.
@@ -46,9 +47,15 @@ def _vq_natural(vq_t, N):
 
 
 def _assert_close(out_gpu, out_orc, v):
-    scale = np.maximum(1.0, v.astype(np.float64).std(axis=2, keepdims=True))
-    err = np.abs(out_gpu.astype(np.float64) - out_orc) / scale
+    """Raw errors within the stated bounds, and (implied by it, since the
+    scale is at least 1) the errors divided by max(1, std of the value
+    channel) as well."""
+    raw = np.abs(out_gpu.astype(np.float64) - out_orc)
     assert np.isfinite(out_gpu).all()
+    assert raw.max() <= MAX_ABS, "raw max-abs %.3g" % raw.max()
+    assert raw.mean() <= MEAN_ABS, "raw mean-abs %.3g" % raw.mean()
+    scale = np.maximum(1.0, v.astype(np.float64).std(axis=2, keepdims=True))
+    err = raw / scale
     assert err.max() <= MAX_ABS, "max-abs %.3g" % err.max()
     assert err.mean() <= MEAN_ABS, "mean-abs %.3g" % err.mean()
     return err
@@ -340,8 +347,10 @@ def test_attention_full_size(name, variant):
             want.append(o[0])
             got.append(out.reshape(BH, w.N, w.d)[bh, r])
         vs.append(np.broadcast_to(inp["v"].reshape(BH, w.N, w.d)[bh].std(axis=0), (len(rows), w.d)))
+    raw = np.abs(np.array(got) - np.array(want))
+    assert raw.max() <= MAX_ABS and raw.mean() <= MEAN_ABS, ("raw", raw.max(), raw.mean())
     scale = np.maximum(1.0, np.concatenate(vs))
-    err = np.abs(np.array(got) - np.array(want)) / scale
+    err = raw / scale
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
 
 

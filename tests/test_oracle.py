@@ -80,6 +80,28 @@ def test_scores_match_sign_matmul(oracle):
         assert np.all(np.abs(z) <= d) and np.all((z - d) % 2 == 0)
 
 
+def test_scores_rows_match_sign_matmul(oracle):
+    """KD1 scores for a chosen block of query rows (the routine the full-size
+    score checks use) pinned to a numpy matmul of the +-1 sign matrices, with
+    rows out of order and repeated, and to the whole-matrix routine."""
+    rng = _rng(17)
+    for d in (1, 33, 64, 72, 128):
+        N = 53
+        q = rng.standard_normal((N, d)).astype(np.float32)
+        k = rng.standard_normal((N, d)).astype(np.float32)
+        q[3, 0] = 0.0
+        k[5, -1] = -0.0
+        bq, _ = oracle.pack(q)
+        bk, _ = oracle.pack(k)
+        rows = np.array([40, 0, 52, 7, 7, 19, 0], np.int32)
+        z = oracle.scores_rows(bq, bk, d, rows)
+        sq = np.where(q >= 0, 1, -1).astype(np.int64)
+        sk = np.where(k >= 0, 1, -1).astype(np.int64)
+        np.testing.assert_array_equal(z, (sq @ sk.T)[rows])
+        np.testing.assert_array_equal(z, oracle.scores(bq[None], bk[None], d)[0][rows])
+        assert z.shape == (len(rows), N) and z.dtype == np.int32
+
+
 def test_scores_sign_flip_invariance(oracle):
     """Negating both Q and K (inputs without zeros) leaves every z unchanged."""
     rng = _rng(8)
