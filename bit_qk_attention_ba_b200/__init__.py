@@ -42,6 +42,21 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _call(device, fn, *args):
+    """Call a libba entry point with `device` current: the library looks up
+    its per-device state (status word, SM count, static scratch) on the
+    current device, and rejects a stream that belongs to another one."""
+    torch = _torch()
+    with torch.cuda.device(device):
+        N.call(fn, *args)
+
+
+def _same_device(*ts):
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError("all tensors must be on one CUDA device, got %s" % sorted(map(str, devs)))
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -65,7 +80,8 @@ def pack_qk(x, bits=None, mu=None):
         bits = torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=x.device)
     if mu is None:
         mu = torch.empty((B, H, Nn), dtype=torch.float32, device=x.device)
-    N.call("ba_pack_qk", _p(x), _dt(x), B, H, Nn, d, _p(bits), _p(mu), _stream(x.device))
+    _same_device(x, bits, mu)
+    _call(x.device, "ba_pack_qk", _p(x), _dt(x), B, H, Nn, d, _p(bits), _p(mu), _stream(x.device))
     return bits, mu
 
 
@@ -78,7 +94,8 @@ def quant_v(v, vq=None, sv=None):
         vq = torch.empty((B, H, d, vq_ld(Nn)), dtype=torch.int8, device=v.device)
     if sv is None:
         sv = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
-    N.call("ba_quant_v", _p(v), _dt(v), B, H, Nn, d, _p(vq), _p(sv), _stream(v.device))
+    _same_device(v, vq, sv)
+    _call(v.device, "ba_quant_v", _p(v), _dt(v), B, H, Nn, d, _p(vq), _p(sv), _stream(v.device))
     return vq, sv
 
 
@@ -100,8 +117,9 @@ def prepass_qkv(q, k, v, outs=None):
                 torch.empty((B, H, d, vq_ld(Nn)), dtype=torch.int8, device=dev),
                 torch.empty((B, H, d), dtype=torch.float32, device=dev))
     bq, muq, bk, muk, vq, sv = outs
-    N.call("ba_prepass_qkv", _p(q), _p(k), _p(v), _dt(q), B, H, Nn, d, _p(bq), _p(muq), _p(bk), _p(muk),
-           _p(vq), _p(sv), _stream(q.device))
+    _same_device(q, k, v, *outs)
+    _call(q.device, "ba_prepass_qkv", _p(q), _p(k), _p(v), _dt(q), B, H, Nn, d, _p(bq), _p(muq), _p(bk),
+          _p(muk), _p(vq), _p(sv), _stream(q.device))
     return outs
 
 
@@ -158,8 +176,9 @@ def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NO
     else:
         _need_cuda(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    N.call("ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
-           B, H, Nn, d, _p(workspace), ws_bytes, _p(out), _dt(out), int(variant), _stream(muq.device))
+    _same_device(bq, muq, bk, muk, vq, sv, out, workspace, bias)
+    _call(muq.device, "ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld,
+          gh, gw, B, H, Nn, d, _p(workspace), ws_bytes, _p(out), _dt(out), int(variant), _stream(muq.device))
     return out
 
 
@@ -173,8 +192,9 @@ def attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA
     if out is None:
         out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=muq.device)
     kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
-    N.call("ba_attention_fwd_noalloc", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw,
-           B, H, Nn, d, _p(out), _dt(out), _stream(muq.device))
+    _same_device(bq, muq, bk, muk, vq, sv, out, bias)
+    _call(muq.device, "ba_attention_fwd_noalloc", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld,
+          gh, gw, B, H, Nn, d, _p(out), _dt(out), _stream(muq.device))
     return out
 
 
@@ -185,7 +205,8 @@ def scores_debug(bq, bk, d, z=None):
     B, H, Nn, _ = bq.shape
     if z is None:
         z = torch.empty((B, H, Nn, Nn), dtype=torch.int32, device=bq.device)
-    N.call("ba_scores_debug", _p(bq), _p(bk), B, H, Nn, d, _p(z), _stream(bq.device))
+    _same_device(bq, bk, z)
+    _call(bq.device, "ba_scores_debug", _p(bq), _p(bk), B, H, Nn, d, _p(z), _stream(bq.device))
     return z
 
 
@@ -216,15 +237,17 @@ def attention_decode(bq, muq, bk, muk, vq, sv, d, bias=None, out=None, out_dtype
     if bias is not None:
         _need_cuda(bias)
         bp, ld = _p(bias), int(bias.shape[-1])
-    N.call("ba_attention_decode", _p(bq), _p(muq), Nq, _p(bk), _p(muk), _p(vq), _p(sv), Nk, bp, ld, B, H, d,
-           _p(workspace), workspace.numel(), _p(out), _dt(out), _stream(muq.device))
+    _same_device(bq, muq, bk, muk, vq, sv, out, workspace, bias)
+    _call(muq.device, "ba_attention_decode", _p(bq), _p(muq), Nq, _p(bk), _p(muk), _p(vq), _p(sv), Nk, bp, ld, B,
+          H, d, _p(workspace), workspace.numel(), _p(out), _dt(out), _stream(muq.device))
     return out
 
 
 def decode_workspace(B, H, nq, nk, d, device=None):
     """A workspace tensor for attention_decode."""
     torch = _torch()
-    nb = int(N.lib().ba_attention_decode_workspace_bytes(B, H, nq, nk, d))
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        nb = int(N.lib().ba_attention_decode_workspace_bytes(B, H, nq, nk, d))
     if nb < 0:
         raise ValueError("invalid decode sizes (1 <= Nq <= 16, d <= 128) or no CUDA device")
     return torch.empty((max(nb, 256),), dtype=torch.uint8, device=device)
@@ -232,8 +255,11 @@ def decode_workspace(B, H, nq, nk, d, device=None):
 
 def check_device_status(device=None) -> int:
     """Synchronise and return the device status word (0 = no kernel failure)."""
+    torch = _torch()
     code = ctypes.c_int(0)
-    st = N.lib().ba_check_device_status(_stream(device), ctypes.byref(code))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        st = N.lib().ba_check_device_status(_stream(dev), ctypes.byref(code))
     if st not in (N.BA_OK, N.BA_ERR_DEVICE_STATUS):
         N.check("ba_check_device_status", st)
     return code.value

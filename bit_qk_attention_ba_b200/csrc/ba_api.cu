@@ -98,6 +98,20 @@ static uintptr_t esize(ba_dtype dt) { return dt == BA_BF16 ? 2 : 4; }
 
 static ba_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BA_OK : BA_ERR_CUDA; }
 
+// The stream must belong to the current device: the status word, the SM
+// count and any library scratch are looked up on the current device, so work
+// queued on another device's stream would get the wrong ones.
+// BA_ERR_CUDA when the runtime cannot say (no device), BA_ERR_INVALID_ARG
+// when the stream belongs to another device.  Checked after every host-only
+// argument check, just before work is queued.
+ba_status check_stream(void* stream)
+{
+    int cur = 0, sdev = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return BA_ERR_CUDA;
+    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) return BA_ERR_CUDA;
+    return sdev == cur ? BA_OK : BA_ERR_INVALID_ARG;
+}
+
 static bool bias_ok(int kind, const float* bias, int64_t ld, int gh, int gw, int N)
 {
     if (kind == BA_BIAS_NONE) return true;
@@ -107,6 +121,20 @@ static bool bias_ok(int kind, const float* bias, int64_t ld, int gh, int gw, int
     if (kind == BA_BIAS_RELPOS2D_CLS)
         return ptr_ok(bias, 4) && gh >= 1 && gw >= 1 && (int64_t)gh * gw + 1 == N;
     return false;
+}
+
+// Every host-side check of the fused forward's arguments except the
+// workspace size (which depends on the path taken).
+ba_status validate_fwd(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                       const int8_t* vq, const float* sv, int bias_kind, const float* bias, int64_t bias_ld,
+                       int grid_h, int grid_w, int B, int H, int N, int d, const void* out, ba_dtype out_dt)
+{
+    if (!sizes_ok(B, H, N, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
+        !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)))
+        return BA_ERR_INVALID_ARG;
+    if (!bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N)) return BA_ERR_INVALID_ARG;
+    return BA_OK;
 }
 
 }  // namespace ba
@@ -136,6 +164,7 @@ ba_status ba_pack_qk(const void* x, ba_dtype dt, int B, int H, int N, int d,
 {
     if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
     if (!ptr_ok(x, esize(dt)) || !ptr_ok(bits, 4) || !ptr_ok(mu, 4)) return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
     const int sms = sm_count();
     if (sms <= 0) return BA_ERR_CUDA;
     return from_cuda(launch_pack(x, dt, (int64_t)B * H * N, d, bits, mu,
@@ -147,6 +176,7 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
 {
     if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
     if (!ptr_ok(v, esize(dt)) || !ptr_ok(vq, 16) || !ptr_ok(sv, 4)) return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
     return from_cuda(launch_quant_v(v, dt, B, H, N, d, vq, sv, static_cast<cudaStream_t>(stream)));
 }
 
@@ -158,6 +188,7 @@ ba_status ba_prepass_qkv(const void* q, const void* k, const void* v, ba_dtype d
     if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
         !ptr_ok(sv, 4))
         return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
     const int sms = sm_count();
     if (sms <= 0) return BA_ERR_CUDA;
     return from_cuda(launch_prepass(q, k, v, dt, B, H, N, d, bq, muq, bk, muk, vq, sv,
@@ -175,6 +206,7 @@ ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk, int B, int H, 
 {
     if (!sizes_ok(B, H, N, d)) return BA_ERR_INVALID_ARG;
     if (!ptr_ok(bq, 4) || !ptr_ok(bk, 4) || !ptr_ok(z, 4)) return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
     if (ceil_div(N, 64) > 65535) return BA_ERR_UNSUPPORTED;
     return from_cuda(launch_scores(bq, bk, B, H, N, d, z, static_cast<cudaStream_t>(stream)));
 }
@@ -198,15 +230,20 @@ ba_status ba_attention_fwd_variant(const uint32_t* bq, const float* muq,
                                    void* workspace, int64_t workspace_bytes,
                                    void* out, ba_dtype out_dt, int variant, void* stream)
 {
-    if (!sizes_ok(B, H, N, d) || (out_dt != BA_F32 && out_dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    const ba_status v = validate_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w, B, H, N, d,
+                                     out, out_dt);
+    if (v != BA_OK) return v;
     if (workspace_bytes < 0 || (workspace_bytes > 0 && !ptr_ok(workspace, 256))) return BA_ERR_INVALID_ARG;
-    if (!ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) || !ptr_ok(muk, 4) || !ptr_ok(vq, 16) ||
-        !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)))
-        return BA_ERR_INVALID_ARG;
-    if (!bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N)) return BA_ERR_INVALID_ARG;
     if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_MMA_B1 && variant != BA_QK_TC_I8 &&
         variant != BA_QK_TC_F8)
         return BA_ERR_INVALID_ARG;
+    const bool ws_needed = variant != BA_QK_MMA_B1 && variant != BA_QK_POPC &&
+                           attn_tc_supports(bias_kind, grid_h, grid_w, N, d);
+    if (ws_needed && workspace_bytes < attn_tc_workspace_bytes(B, H, N, d, bias_kind, grid_h, grid_w))
+        return BA_ERR_INVALID_ARG;
+    if (variant != BA_QK_AUTO && variant != BA_QK_POPC && variant != BA_QK_MMA_B1 && !ws_needed)
+        return BA_ERR_UNSUPPORTED;
+    if (const ba_status e = check_stream(stream)) return e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (variant == BA_QK_MMA_B1)
         return from_cuda(launch_attn_b1(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h,
@@ -266,6 +303,7 @@ ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
         !ptr_ok(sv, 4) || !ptr_ok(out, esize(out_dt)) || !ptr_ok(workspace, 256))
         return BA_ERR_INVALID_ARG;
     if (bias != nullptr && (!ptr_ok(bias, 4) || bias_ld < Nk)) return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
     const int sms = sm_count();
     if (sms <= 0) return BA_ERR_CUDA;
     if (workspace_bytes < attn_decode_workspace_bytes(B, H, Nk, d, sms)) return BA_ERR_INVALID_ARG;

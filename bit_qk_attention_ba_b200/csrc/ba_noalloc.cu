@@ -13,6 +13,10 @@
 namespace ba {
 
 int64_t attn_tc_workspace_bytes(int B, int H, int N, int d, int bias_kind, int gh, int gw);
+ba_status validate_fwd(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                       const int8_t* vq, const float* sv, int bias_kind, const float* bias, int64_t bias_ld,
+                       int grid_h, int grid_w, int B, int H, int N, int d, const void* out, ba_dtype out_dt);
+ba_status check_stream(void* stream);
 
 namespace {
 
@@ -47,9 +51,15 @@ extern "C" ba_status ba_attention_fwd_noalloc(const uint32_t* bq, const float* m
                                               int B, int H, int N, int d,
                                               void* out, ba_dtype out_dt, void* stream)
 {
+    // The same argument checks as ba_attention_fwd, before the static array
+    // is looked up (which loads this file's module on first use).
+    const ba_status v = ba::validate_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w, B, H,
+                                         N, d, out, out_dt);
+    if (v != BA_OK) return v;
     const int64_t need = ba_attention_workspace_bytes(B, H, N, d, bias_kind, grid_h, grid_w);
     if (need < 0) return BA_ERR_INVALID_ARG;
     if (need > ba::kStaticScratchBytes) return BA_ERR_UNSUPPORTED;
+    if (const ba_status e = ba::check_stream(stream)) return e;
     void* scratch = nullptr;
     if (need > 0) {
         scratch = ba::static_scratch();

@@ -21,6 +21,11 @@
  *     void*; NULL is the legacy default stream).
  *   - Arguments are validated before anything is queued; an invalid call
  *     returns BA_ERR_INVALID_ARG (or BA_ERR_UNSUPPORTED) and queues nothing.
+ *   - Work runs on the CURRENT device: the library's per-device state (status
+ *     word, SM count, the static scratch of ba_attention_fwd_noalloc) is that
+ *     of the device current on the calling thread, and `stream` must belong
+ *     to it (BA_ERR_INVALID_ARG otherwise; BA_ERR_CUDA when the runtime has
+ *     no device).  The buffers must live on that device too.
  *   - A launch failure reported by the CUDA runtime returns BA_ERR_CUDA.
  *   - Kernels that wait on hardware barriers give up after a bounded number of
  *     polls, record a code in a device status word and exit cleanly;

@@ -61,17 +61,27 @@ def test_noalloc_matches_workspace_path_and_oracle(w):
     bk, muk = ba.pack_qk(k)
     vq, sv = ba.quant_v(v)
     ref = ba.attention_fwd(bq, muq, bk, muk, vq, sv, w.d, bias=bias, bias_kind=kind, ld=inp["ld"], grid=w.grid)
-    out = torch.empty_like(ref)
+    outs = [torch.full_like(ref, float("nan")) for _ in range(2)]
     torch.cuda.synchronize()
-    before = torch.cuda.memory_allocated(dev)
-    ba.attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, w.d, bias=bias, bias_kind=kind, ld=inp["ld"],
-                             grid=w.grid, out=out)
+    run = lambda o: ba.attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, w.d, bias=bias, bias_kind=kind,
+                                             ld=inp["ld"], grid=w.grid, out=o)
+    # First call: may load the module that holds the static array.
+    run(outs[0])
     torch.cuda.synchronize()
-    assert torch.cuda.memory_allocated(dev) == before          # nothing allocated through torch
+    # Second call, right after: no allocation through torch, and no device
+    # memory taken by the library itself (cudaMemGetInfo before and after).
+    before_torch = torch.cuda.memory_allocated(dev)
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    run(outs[1])
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info(dev)
+    assert torch.cuda.memory_allocated(dev) == before_torch
+    assert free_after == free_before
     assert ba.check_device_status() == 0
-    # same kernels, same staging: identical bits
-    assert torch.equal(out, ref)
     gh, gw = w.grid
     orc = O.forward(inp["q"], inp["k"], inp["v"], kind, inp["bias"], inp["ld"], gh, gw)["out"]
-    err = np.abs(out.cpu().numpy().astype(np.float64) - orc)
-    assert err.max() <= 2e-2 and err.mean() <= 2e-3
+    for out in outs:
+        # same kernels, same staging: identical bits to the workspace path
+        assert torch.equal(out, ref)
+        err = np.abs(out.cpu().numpy().astype(np.float64) - orc)
+        assert err.max() <= 2e-2 and err.mean() <= 2e-3
