@@ -38,6 +38,10 @@ from bit_qk_attention_ba_b200.workloads import (BIAS_KIND, DECODE_WORKLOADS, WOR
                                                 make_decode_inputs, make_inputs)
 
 METRIC = "binary attention effective TOPS (4*B*H*N^2*d per step)"
+DTYPE = ("+-1 int8 QK on tcgen05 kind::i8 (s32 accumulate), u8 x s8 PV on tcgen05 kind::i8 (s32), "
+         "fp32 scores and softmax")
+# The gate workloads reported beside the headline one, each timed on its own.
+SIDE_WORKLOADS = ("deit_b384", "deit_s", "dit_xl2", "deit_t")
 L2_BYTES = 126 * 2 ** 20
 CSRC = os.path.join(ROOT, "bit_qk_attention_ba_b200", "csrc")
 
@@ -81,6 +85,35 @@ def attn_bytes(w, out_bytes):
         gh, gw = w.grid
         b += w.H * ((2 * gh - 1) * (2 * gw - 1) + (3 if w.bias == "relpos2d_cls" else 0)) * 4
     return b
+
+
+def roofline(w, attn_t, out_bytes, variant):
+    """Roofline of the fused attention call timed in isolation (CUDA events
+    around ba_attention_fwd): tensor-bound when ops / int8 peak exceeds
+    algorithmic bytes / HBM peak.  The int8 peak is 2 x the measured bf16 GEMM
+    rate (the nominal B200 int8 : bf16 ratio), the burst figure since the call
+    is timed alone; the fraction of the sustained figure is given beside it."""
+    pk = peaks()
+    int8_burst, int8_sus = 2.0 * pk["bf16"], 2.0 * pk["bf16_sus"]
+    abytes = attn_bytes(w, out_bytes)
+    t_tensor, t_hbm = w.ops / (int8_burst * 1e12), abytes / (pk["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = w.ops / attn_t / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": int8_burst, "unit": "TOPS",
+                "frac": ach / int8_burst, "frac_sustained": ach / int8_sus,
+                "peak_source": "int8 = 2 x measured burst bf16 GEMM (%s); frac_sustained against 2 x the "
+                               "sustained bf16 figure" % pk["src"]}
+    else:
+        ach = abytes / attn_t / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "peak_source": "measured HBM copy (%s)" % pk["src"]}
+    kname, ksrc = attn_kernel(w, variant)
+    roof["kernel"] = kname
+    roof["traffic"] = recorded_traffic(kname, ksrc, w.name)
+    roof["kernel_us"] = attn_t * 1e6
+    roof["algorithmic_bytes"] = abytes
+    roof["ops"] = w.ops
+    return roof
 
 
 def _code_only(text):
@@ -214,6 +247,57 @@ def max_over_ranks(x, world, device=None):
 
 
 # ------------------------------------------------------------------ our arm
+
+def time_side_workload(w, variant, dev, steps=50, warmup=10):
+    """A gate workload timed on its own: the pre-pass + attention step and the
+    attention call alone (CUDA events, median over the timed steps, the L2
+    flushed between steps when the inputs fit in it)."""
+    import torch
+    import bit_qk_attention_ba_b200 as ba
+    inp = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v = (torch.from_numpy(inp[n]).to(tdt).to(dev) for n in ("q", "k", "v"))
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
+    kind, ld, grid = BIAS_KIND[w.bias], inp["ld"], w.grid
+    pre = ba.prepass_qkv(q, k, v)
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=tdt, device=dev)
+    ws = ba.attention_workspace(w.B, w.H, w.N, w.d, kind, grid, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + (bias.numel() * 4 if bias is not None else 0)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes < 2 * L2_BYTES else None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        ba.prepass_qkv(q, k, v, pre)
+        if e is not None:
+            e[1].record(stream)
+        ba.attention_fwd(*pre, w.d, bias=bias, bias_kind=kind, ld=ld, grid=grid, out=out, variant=variant,
+                         workspace=ws)
+        if e is not None:
+            e[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        step(ev[i])
+    torch.cuda.synchronize(dev)
+    step_ms = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
+    attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    roof = roofline(w, attn_ms * 1e-3, 2 if tdt == torch.bfloat16 else 4, variant)
+    status = ba.check_device_status(dev)
+    del q, k, v, bias, pre, out, ws, flush
+    torch.cuda.empty_cache()
+    return {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": w.bias, "attention_us": attn_ms * 1e3,
+            "step_us": step_ms * 1e3, "step_tops": w.ops / (step_ms * 1e-3) / 1e12,
+            "attention_tops": w.ops / (attn_ms * 1e-3) / 1e12, "steps": steps, "warmup": warmup,
+            "l2": "flushed between steps" if in_bytes < 2 * L2_BYTES else "inputs larger than L2",
+            "roofline": roof, "device_status": status}
+
 
 def run_ours(args, w, rank, local_rank, world):
     import torch
@@ -350,30 +434,15 @@ def run_ours(args, w, rank, local_rank, world):
     fast_rp = kind == NAT.BA_BIAS_RELPOS2D and grid and grid[1] % 128 == 0
     launches_per_step = ba.prepass_launches(w.N, d, tdt) + (1 + (1 if fast_rp else 0) if tc_path else 0) + 1
     value = aggregate_tops(world, ops, ms)
-    pk = peaks()
     attn_t = statistics.median(attn_ms) * 1e-3
-    int8_peak = (pk["bf16_sus"]) * 2.0          # int8 dense = 2x bf16 dense (nominal ratio)
-    abytes = attn_bytes(w, out_bytes)
-    t_tensor, t_hbm = ops / (int8_peak * 1e12), abytes / (pk["hbm_gbs"] * 1e9)
-    if t_tensor >= t_hbm:
-        roof = {"bound": "tensor", "achieved": ops / attn_t / 1e12, "peak": int8_peak, "unit": "TOPS"}
-    else:
-        roof = {"bound": "hbm", "achieved": abytes / attn_t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    kname, ksrc = attn_kernel(w, args.variant)
-    roof["kernel"] = kname
-    roof["traffic"] = recorded_traffic(kname, ksrc, w.name)
     # CUDA events bracket the whole ba_attention_fwd call: the key staging
     # pre-passes plus the fused kernel (the staging is the small remainder).
-    roof["kernel_us"] = attn_t * 1e6
-    roof["peak_source"] = ("int8 = 2 x measured sustained bf16 (%s)" % pk["src"]) if roof["bound"] == "tensor" \
-        else "measured HBM copy (%s)" % pk["src"]
-    roof["algorithmic_bytes"] = abytes
+    roof = roofline(w, attn_t, out_bytes, args.variant)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u8/s8/b1 (QK b1, PV u8xs8->s32, softmax fp32)", "data": "synthetic",
+        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
                    "bias": w.bias, "parallelism": "replicas%d" % world,
                    "l2": "flushed between steps" if flush is not None else "inputs larger than L2",
@@ -386,6 +455,13 @@ def run_ours(args, w, rank, local_rank, world):
         "clocks": clocks,
         "device_status": status,
     }
+    if not args.no_side_workloads:
+        # every rank times the same side workloads, so the ranks stay in step
+        side = {}
+        for name in SIDE_WORKLOADS:
+            if name != w.name:
+                side[name] = time_side_workload(WORKLOADS[name], args.variant, dev)
+        line["workloads"] = side
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
     if world > 1:
@@ -492,7 +568,7 @@ def run_decode(args, w, rank, local_rank, world):
     line = {
         "metric": METRIC, "value": aggregate_tops(world, w.ops, ms), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "u8/s8/b1 (QK b1 popcount, PV u8xs8->s32, softmax fp32)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "b1 QK by XOR/popcount on CUDA cores, u8 x s8 PV by dp4a (s32), fp32 softmax",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "input_dtype": w.dtype, "bias": "none", "parallelism": "replicas%d" % world,
@@ -633,6 +709,8 @@ def main(argv=None):
     ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 2 mma.sync b1, 3 tcgen05 i8, 4 tcgen05 f8")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side-workloads", action="store_true",
+                    help="skip the gate workloads timed beside the headline one")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
