@@ -7,9 +7,11 @@ product path never does, and the two share no code: this wrapper loads
 
 Source ("BA notes"): the paper-notes page "BinaryAttention: One-Bit
 QK-Attention for Vision and Diffusion Transformers" (CVPR 2026), sections
-Key design 1 (scaled binary Q/K), Key design 2 (bias enhancement) and Key
-design 3 (hybrid 8-bit quantisation of P and V).  Every numeric step lives in
-the C file; this module only marshals numpy arrays.
+Key design 1 (scaled binary Q/K), Key design 2 (bias enhancement), Key
+design 3 (hybrid 8-bit quantisation of P and V) and, for the training-side
+backward pass, Key design 4 (QAT with a straight-through estimator for sign).
+Every numeric step lives in the C file; this module only marshals numpy
+arrays.
 """
 from __future__ import annotations
 
@@ -72,6 +74,11 @@ def _load():
     lib.bao_attention_fwd_rows.restype = i32
     lib.bao_attention_decode.argtypes = [P, P, P, P, P, P, i32, P, i64, i64, i32, i32, i32, i32, P]
     lib.bao_attention_decode.restype = None
+    lib.bao_bwd_core.argtypes = [P, P, P, P, P, P, i32, i32, i32, P, P, P, P, P, P, P, P]
+    lib.bao_bwd_core.restype = None
+    lib.bao_attention_bwd.argtypes = [P, P, P, i32, P, i64, i32, i32, i32, i32, i32, i32, P,
+                                      ctypes.c_double, i32, P, P, P, P, P]
+    lib.bao_attention_bwd.restype = None
     _lib = lib
     return lib
 
@@ -232,3 +239,43 @@ def forward(q, k, v, bias_kind=BIAS_NONE, bias=None, ld=0, gh=0, gw=0, nthreads=
     out, used = attention_fwd(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw, B, H, d, nthreads)
     return dict(bits_q=bq, mu_q=muq, bits_k=bk, mu_k=muk, vq=vq, sv=sv,
                 out=out.reshape(B, H, N, d), threads=used)
+
+
+def bwd_core(s, t, muq, muk, vh, bias, dO, quantise_p=False):
+    """The differentiable core of one head (Key design 4 backward, see the C
+    file): continuous s, t, vh [N, d], muq, muk [N], bias [N, N] or None,
+    dO [N, d].  Returns dict O, ds, dt, dvh, dmuq, dmuk, dbias (float64)."""
+    s, t, vh, dO = (_c(a, np.float64) for a in (s, t, vh, dO))
+    muq, muk = _c(muq, np.float64), _c(muk, np.float64)
+    b = None if bias is None else _c(bias, np.float64)
+    N, d = s.shape
+    out = {k: np.zeros((N, d)) for k in ("O", "ds", "dt", "dvh")}
+    out["dmuq"], out["dmuk"] = np.zeros(N), np.zeros(N)
+    out["dbias"] = np.zeros((N, N)) if b is not None else None
+    _load().bao_bwd_core(_ptr(s), _ptr(t), _ptr(muq), _ptr(muk), _ptr(vh), _ptr(b), N, d, int(bool(quantise_p)),
+                         _ptr(dO), _ptr(out["O"]), _ptr(out["ds"]), _ptr(out["dt"]), _ptr(out["dvh"]),
+                         _ptr(out["dmuq"]), _ptr(out["dmuk"]), _ptr(out["dbias"]))
+    return out
+
+
+def attention_bwd(q, k, v, dO, bias_kind=BIAS_NONE, bias=None, ld=0, gh=0, gw=0, ste_clip=float("inf"),
+                  quantise=True):
+    """Backward with straight-through estimators from raw q, k, v [B, H, N, d]
+    and dO [B, H, N, d].  Returns dict dq, dk, dv, O [B, H, N, d] and dbias
+    (dense [H, N, ld], or the rel-pos table's shape [H, G (+3)], or None)."""
+    B, H, N, d = q.shape
+    q, k, v = (_c(a, np.float32) for a in (q, k, v))
+    dO = _c(dO, np.float64)
+    b = None if bias is None else _c(bias, np.float32)
+    res = {n: np.zeros((B, H, N, d)) for n in ("dq", "dk", "dv", "O")}
+    db = None
+    if bias_kind == BIAS_DENSE:
+        db = np.zeros((H, N, ld))
+    elif bias_kind in (BIAS_RELPOS2D, BIAS_RELPOS2D_CLS):
+        G = (2 * gh - 1) * (2 * gw - 1) + (3 if bias_kind == BIAS_RELPOS2D_CLS else 0)
+        db = np.zeros((H, G))
+    _load().bao_attention_bwd(_ptr(q), _ptr(k), _ptr(v), bias_kind, _ptr(b), int(ld), gh, gw, B, H, N, d,
+                              _ptr(dO), float(ste_clip), int(bool(quantise)), _ptr(res["dq"]), _ptr(res["dk"]),
+                              _ptr(res["dv"]), _ptr(res["O"]), _ptr(db))
+    res["dbias"] = db
+    return res

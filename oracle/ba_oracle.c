@@ -1,5 +1,6 @@
 /*
- * ba_oracle.c -- plain CPU oracle for the BinaryAttention forward pass.
+ * ba_oracle.c -- plain CPU oracle for the BinaryAttention forward pass and its
+ * training-side backward pass (straight-through estimators).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * CPU-baseline leg of the benchmark may load this library.  The product path
@@ -369,4 +370,238 @@ int bao_attention_fwd(const uint32_t* bq, const double* muq,
 {
     return bao_attention_fwd_rows(bq, muq, bk, muk, vq, sv, bias_kind, bias, ld, gh, gw,
                                   (int64_t)B * H, H, N, d, 0, N, out, nthreads);
+}
+
+/* ---- training side: the backward pass with straight-through estimators ----
+ *
+ * Source: Key design 4 of the BA notes (QAT + self-distillation; "Loss and
+ * training strategy"): training applies sign quantisation to Q and K in the
+ * forward pass and approximates its gradient in the backward pass with a
+ * straight-through estimator (STE).  The page says nothing more, so the
+ * readings taken here (also listed in the design notes) are:
+ *   - every quantiser passes its gradient straight through: sign(x) (optionally
+ *     clipped, d sign(x)/dx := [|x| <= clip], clip = +inf for the plain
+ *     identity), the u8 rounding of P~ and the int8 rounding of V;
+ *   - everything else is differentiated exactly: the per-token scale
+ *     mu = mean |x| (d mu / d x_c = sign(x_c) / d, with sign(0) = +1 as in the
+ *     forward), the product with sqrt(d), the bias, the softmax;
+ *   - the row maximum m is a constant of the backward (softmax is invariant
+ *     to it), as in FlashAttention-style backward passes;
+ *   - with pq the rounded codes, the forward is O = (pq / 255) V^ / l with
+ *     l = sum_j P~ unquantised, so reverse-mode differentiation gives
+ *       dV^_j = sum_i P^_ij dO_i                  (P^ = pq / (255 l))
+ *       dS_ij = P_ij (dO_i . V^_j - dO_i . O_i)   (P = P~ / l, O the forward output)
+ *     the quantised P^ where the product used it, the unquantised softmax
+ *     Jacobian through the straight-through rounding.
+ * Chain to the inputs (KD2: S = mu_q mu_k s.t / sqrt(d) + b):
+ *   dz_ij   = dS_ij mu_q,i mu_k,j / sqrt(d)
+ *   dmu_q,i = sum_j dS_ij mu_k,j z_ij / sqrt(d);  dmu_k,j likewise over i
+ *   ds_i    = sum_j dz_ij t_j;   dt_j = sum_i dz_ij s_i
+ *   dq_ic   = ds_ic [|q_ic| <= clip] + dmu_q,i sign(q_ic) / d;  dk likewise
+ *   db_ij  += dS_ij (a bias shared over the batch sums over it)
+ */
+
+/*
+ * The differentiable core for one (batch, head), on continuous inputs:
+ *   S_ij = muq_i muk_j (s_i . t_j) / sqrt(d) + bias_ij,  P~ = exp(S - m),
+ *   l_i = sum_j P~_ij,  O_i = sum_j W_ij vh_j  with W = P~ / l (quantise_p = 0)
+ *   or W = round(255 P~) / (255 l) (quantise_p = 1).
+ * s, t [N, d] and vh [N, d] are arbitrary reals here (for the method s, t are
+ * the +-1 signs and vh the dequantised values); bias [N, N] (row stride N) is
+ * the head's bias, or NULL.  Given dO [N, d] it returns O and the gradients
+ * ds, dt, dvh [N, d], dmuq, dmuk [N] and dbias [N, N] (each may be NULL).
+ */
+void bao_bwd_core(const double* s, const double* t, const double* muq, const double* muk,
+                  const double* vh, const double* bias, int N, int d, int quantise_p,
+                  const double* dO, double* O, double* ds, double* dt, double* dvh,
+                  double* dmuq, double* dmuk, double* dbias)
+{
+    const double rsd = sqrt((double)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)N * N);
+    double* P = (double*)malloc(sizeof(double) * (size_t)N * N);   /* P~ / l */
+    double* W = (double*)malloc(sizeof(double) * (size_t)N * N);   /* what the product used */
+    double* Oi = (double*)malloc(sizeof(double) * (size_t)N * d);
+    double* dS = (double*)malloc(sizeof(double) * (size_t)N * N);
+
+    for (int i = 0; i < N; ++i) {
+        double m = -INFINITY;
+        for (int j = 0; j < N; ++j) {
+            double zz = 0.0;
+            for (int c = 0; c < d; ++c) zz += s[(int64_t)i * d + c] * t[(int64_t)j * d + c];
+            z[(int64_t)i * N + j] = zz;
+            double S = muq[i] * muk[j] * zz / rsd + (bias ? bias[(int64_t)i * N + j] : 0.0);
+            P[(int64_t)i * N + j] = S;
+            if (S > m) m = S;
+        }
+        double l = 0.0;
+        for (int j = 0; j < N; ++j) {
+            double e = exp(P[(int64_t)i * N + j] - m);
+            P[(int64_t)i * N + j] = e;
+            l += e;
+        }
+        for (int j = 0; j < N; ++j) {
+            double e = P[(int64_t)i * N + j];
+            W[(int64_t)i * N + j] = quantise_p ? nearbyint(255.0 * e) / (255.0 * l) : e / l;
+            P[(int64_t)i * N + j] = e / l;
+        }
+        for (int c = 0; c < d; ++c) {
+            double o = 0.0;
+            for (int j = 0; j < N; ++j) o += W[(int64_t)i * N + j] * vh[(int64_t)j * d + c];
+            Oi[(int64_t)i * d + c] = o;
+        }
+    }
+    /* dS_ij = P_ij (dO_i . vh_j - dO_i . O_i) */
+    for (int i = 0; i < N; ++i) {
+        double D = 0.0;
+        for (int c = 0; c < d; ++c) D += dO[(int64_t)i * d + c] * Oi[(int64_t)i * d + c];
+        for (int j = 0; j < N; ++j) {
+            double dp = 0.0;
+            for (int c = 0; c < d; ++c) dp += dO[(int64_t)i * d + c] * vh[(int64_t)j * d + c];
+            dS[(int64_t)i * N + j] = P[(int64_t)i * N + j] * (dp - D);
+        }
+    }
+    if (O) memcpy(O, Oi, sizeof(double) * (size_t)N * d);
+    if (dvh)
+        for (int j = 0; j < N; ++j)
+            for (int c = 0; c < d; ++c) {
+                double g = 0.0;
+                for (int i = 0; i < N; ++i) g += W[(int64_t)i * N + j] * dO[(int64_t)i * d + c];
+                dvh[(int64_t)j * d + c] = g;
+            }
+    if (dbias)
+        for (int64_t e = 0; e < (int64_t)N * N; ++e) dbias[e] = dS[e];
+    if (dmuq)
+        for (int i = 0; i < N; ++i) {
+            double g = 0.0;
+            for (int j = 0; j < N; ++j) g += dS[(int64_t)i * N + j] * muk[j] * z[(int64_t)i * N + j] / rsd;
+            dmuq[i] = g;
+        }
+    if (dmuk)
+        for (int j = 0; j < N; ++j) {
+            double g = 0.0;
+            for (int i = 0; i < N; ++i) g += dS[(int64_t)i * N + j] * muq[i] * z[(int64_t)i * N + j] / rsd;
+            dmuk[j] = g;
+        }
+    if (ds)
+        for (int i = 0; i < N; ++i)
+            for (int c = 0; c < d; ++c) {
+                double g = 0.0;
+                for (int j = 0; j < N; ++j)
+                    g += dS[(int64_t)i * N + j] * muq[i] * muk[j] / rsd * t[(int64_t)j * d + c];
+                ds[(int64_t)i * d + c] = g;
+            }
+    if (dt)
+        for (int j = 0; j < N; ++j)
+            for (int c = 0; c < d; ++c) {
+                double g = 0.0;
+                for (int i = 0; i < N; ++i)
+                    g += dS[(int64_t)i * N + j] * muq[i] * muk[j] / rsd * s[(int64_t)i * d + c];
+                dt[(int64_t)j * d + c] = g;
+            }
+    free(z); free(P); free(W); free(Oi); free(dS);
+}
+
+/*
+ * The whole backward with straight-through estimators, from the raw inputs:
+ *   q, k, v [BH, N, d] fp32 values; bias as for bao_bias_value (kind 0..3);
+ *   dO [BH, N, d].  quantise = 1 runs the method (sign Q/K, u8 P, int8 V);
+ *   quantise = 0 keeps the sign of Q/K but uses P unrounded and V itself.
+ *   ste_clip: the sign's gradient passes where |x| <= ste_clip (+inf: always).
+ * Outputs dq, dk, dv [BH, N, d]; O [BH, N, d] (the forward output, may be
+ * NULL); dbias (may be NULL): dense [H, N, ld] (entries j >= N untouched), or
+ * for the relative-position kinds the table's shape [H, G (+3)] -- summed
+ * over the batch and over every (i, j) that reads an entry.  dbias is
+ * overwritten.
+ */
+void bao_attention_bwd(const float* q, const float* k, const float* v,
+                       int bias_kind, const float* bias, int64_t ld, int gh, int gw,
+                       int B, int H, int N, int d, const double* dO,
+                       double ste_clip, int quantise,
+                       double* dq, double* dk, double* dv, double* O, double* dbias)
+{
+    const int64_t BH = (int64_t)B * H;
+    const size_t Nd = (size_t)N * d;
+    double* s = (double*)malloc(sizeof(double) * Nd);
+    double* t = (double*)malloc(sizeof(double) * Nd);
+    double* vh = (double*)malloc(sizeof(double) * Nd);
+    double* muq = (double*)malloc(sizeof(double) * (size_t)N);
+    double* muk = (double*)malloc(sizeof(double) * (size_t)N);
+    double* b = bias_kind ? (double*)malloc(sizeof(double) * (size_t)N * N) : NULL;
+    double* ds = (double*)malloc(sizeof(double) * Nd);
+    double* dt = (double*)malloc(sizeof(double) * Nd);
+    double* dmuq = (double*)malloc(sizeof(double) * (size_t)N);
+    double* dmuk = (double*)malloc(sizeof(double) * (size_t)N);
+    double* db = bias_kind ? (double*)malloc(sizeof(double) * (size_t)N * N) : NULL;
+    int8_t* vq = (int8_t*)malloc(Nd);
+    float* sv = (float*)malloc(sizeof(float) * (size_t)d);
+
+    if (dbias && bias_kind) {
+        int64_t per_head = 0;
+        if (bias_kind == 1) per_head = (int64_t)N * ld;
+        if (bias_kind == 2) per_head = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+        if (bias_kind == 3) per_head = (int64_t)(2 * gh - 1) * (2 * gw - 1) + 3;
+        for (int64_t e = 0; e < (int64_t)H * per_head; ++e) dbias[e] = 0.0;
+    }
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % H);
+        const float* qh = q + bh * (int64_t)Nd;
+        const float* kh = k + bh * (int64_t)Nd;
+        const float* vhd = v + bh * (int64_t)Nd;
+        for (int i = 0; i < N; ++i) {
+            double aq = 0.0, ak = 0.0;
+            for (int c = 0; c < d; ++c) {
+                s[(int64_t)i * d + c] = sign_pm1(qh[(int64_t)i * d + c]);
+                t[(int64_t)i * d + c] = sign_pm1(kh[(int64_t)i * d + c]);
+                aq += fabs((double)qh[(int64_t)i * d + c]);
+                ak += fabs((double)kh[(int64_t)i * d + c]);
+            }
+            muq[i] = aq / d;
+            muk[i] = ak / d;
+        }
+        if (quantise) {
+            bao_quant_v(vhd, 1, N, d, vq, sv);
+            for (size_t e = 0; e < Nd; ++e) vh[e] = (double)sv[e % d] * (double)vq[e];
+        } else {
+            for (size_t e = 0; e < Nd; ++e) vh[e] = (double)vhd[e];
+        }
+        if (b)
+            for (int i = 0; i < N; ++i)
+                for (int j = 0; j < N; ++j)
+                    b[(int64_t)i * N + j] = bao_bias_value(bias_kind, bias, ld, h, N, gh, gw, i, j);
+        bao_bwd_core(s, t, muq, muk, vh, b, N, d, quantise, dO + bh * (int64_t)Nd,
+                     O ? O + bh * (int64_t)Nd : NULL, ds, dt, dv + bh * (int64_t)Nd, dmuq, dmuk, db);
+        for (int i = 0; i < N; ++i)
+            for (int c = 0; c < d; ++c) {
+                const int64_t e = (int64_t)i * d + c;
+                const double xq = qh[e], xk = kh[e];
+                dq[bh * (int64_t)Nd + e] = (fabs(xq) <= ste_clip ? ds[e] : 0.0) + dmuq[i] * s[e] / d;
+                dk[bh * (int64_t)Nd + e] = (fabs(xk) <= ste_clip ? dt[e] : 0.0) + dmuk[i] * t[e] / d;
+            }
+        if (dbias && db) {
+            for (int i = 0; i < N; ++i)
+                for (int j = 0; j < N; ++j) {
+                    const double g = db[(int64_t)i * N + j];
+                    if (bias_kind == 1) {
+                        dbias[((int64_t)h * N + i) * ld + j] += g;
+                    } else if (bias_kind == 2) {
+                        int ri = i / gw, ci = i % gw, rj = j / gw, cj = j % gw;
+                        int64_t G = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+                        dbias[h * G + (int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1)] += g;
+                    } else if (bias_kind == 3) {
+                        int64_t G = (int64_t)(2 * gh - 1) * (2 * gw - 1);
+                        double* tb = dbias + h * (G + 3);
+                        if (i == 0 && j == 0) tb[G + 2] += g;
+                        else if (i == 0) tb[G] += g;
+                        else if (j == 0) tb[G + 1] += g;
+                        else {
+                            int pi = i - 1, pj = j - 1;
+                            int ri = pi / gw, ci = pi % gw, rj = pj / gw, cj = pj % gw;
+                            tb[(int64_t)(ri - rj + gh - 1) * (2 * gw - 1) + (ci - cj + gw - 1)] += g;
+                        }
+                    }
+                }
+        }
+    }
+    free(s); free(t); free(vh); free(muq); free(muk); free(b); free(ds); free(dt);
+    free(dmuq); free(dmuk); free(db); free(vq); free(sv);
 }
