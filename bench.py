@@ -11,9 +11,11 @@ Prints ONE JSON line on rank 0.
 
 Metric: effective TOPS = 4*B*H*N^2*d per step / step time (higher is better);
 ms_per_step and the fused kernel's roofline fraction are reported alongside.
-Multi-GPU (torchrun): every rank runs its own copy of the workload (the (b, h)
-units are independent, no collective on the data path); value = all ranks'
-operations / max-over-ranks time ("scaling": "weak").
+Multi-GPU (torchrun): the job is a global batch of N x B batch elements split
+into contiguous slices of B, one per rank (bit_qk_attention_ba_b200.sharding;
+the (b, h) units are independent, no collective on the data path); rank r's
+slice is drawn with seed + its first global batch index.  value = all ranks'
+operations / max-over-ranks time ("scaling": "weak": the per-GPU work is fixed).
 """
 from __future__ import annotations
 
@@ -34,6 +36,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from bit_qk_attention_ba_b200.sharding import shard_range  # noqa: E402
 from bit_qk_attention_ba_b200.workloads import (BIAS_KIND, DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
                                                 make_decode_inputs, make_inputs)
 
@@ -230,9 +233,30 @@ def dist_env():
 
 
 def aggregate_tops(world, ops_per_rank, ms_per_step):
-    """Whole-job effective TOPS: every rank runs its own copy of the workload
-    (replicas, weak scaling), timed by the slowest rank."""
+    """Whole-job effective TOPS: every rank runs one batch slice of the same
+    size (weak scaling), timed by the slowest rank."""
     return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def input_bytes(w):
+    """Bytes of one step's inputs on the device (q, k, v and the bias)."""
+    es = 2 if w.dtype == "bf16" else 4
+    b = 3 * w.B * w.H * w.N * w.d * es
+    if w.bias == "dense":
+        b += w.H * w.N * w.ld * 4
+    elif w.bias in ("relpos2d", "relpos2d_cls"):
+        gh, gw = w.grid
+        b += w.H * ((2 * gh - 1) * (2 * gw - 1) + (3 if w.bias == "relpos2d_cls" else 0)) * 4
+    return b
+
+
+def bench_config(w, world, variant):
+    """The `config` object of the JSON line, the same for both arms."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
+            "bias": w.bias, "parallelism": "dp%d" % world, "global_batch": world * w.B,
+            "split": "contiguous batch slices of %d per rank, no data-path collective" % w.B,
+            "l2": "flushed between steps" if input_bytes(w) < 2 * L2_BYTES else "inputs larger than L2",
+            "qk_variant": variant}
 
 
 def max_over_ranks(x, world, device=None):
@@ -311,7 +335,10 @@ def run_ours(args, w, rank, local_rank, world):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    inp = make_inputs(w)
+    # this rank's slice of the global batch (world x B elements)
+    lo, hi = shard_range(world * w.B, world, rank)
+    assert hi - lo == w.B
+    inp = make_inputs(w, seed=w.seed + lo)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {n: torch.from_numpy(inp[n]).to(tdt).pin_memory() for n in ("q", "k", "v")}
     q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
@@ -327,6 +354,7 @@ def run_ours(args, w, rank, local_rank, world):
     ws = ba.attention_workspace(w.B, w.H, w.N, d, kind, grid, device=dev)
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + (bias.numel() * 4 if bias is not None else 0)
+    assert in_bytes == input_bytes(w)
     flush = None
     if in_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -443,10 +471,7 @@ def run_ours(args, w, rank, local_rank, world):
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
-                   "bias": w.bias, "parallelism": "replicas%d" % world,
-                   "l2": "flushed between steps" if flush is not None else "inputs larger than L2",
-                   "qk_variant": args.variant},
+        "config": bench_config(w, world, args.variant),
         "roofline": roof,
         "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -477,6 +502,12 @@ def decode_bytes(w, out_bytes):
     output."""
     BH, W = w.B * w.H, (w.d + 31) // 32
     return BH * w.Nk * (W * 4 + 4 + w.d) + BH * w.d * 4 + BH * w.Nq * (W * 4 + 4) + BH * w.Nq * w.d * out_bytes
+
+
+def decode_config(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "input_dtype": w.dtype, "bias": "none", "parallelism": "replicas%d" % world,
+            "l2": "cache larger than L2", "ops": "4*B*H*Nq*Nk*d per step"}
 
 
 def run_decode(args, w, rank, local_rank, world):
@@ -570,9 +601,7 @@ def run_decode(args, w, rank, local_rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "b1 QK by XOR/popcount on CUDA cores, u8 x s8 PV by dp4a (s32), fp32 softmax",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
-                   "input_dtype": w.dtype, "bias": "none", "parallelism": "replicas%d" % world,
-                   "l2": "cache larger than L2", "ops": "4*B*H*Nq*Nk*d per step"},
+        "config": decode_config(w, world),
         "roofline": roof,
         "e2e": {"value": world * w.ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
                 "h2d_bytes_per_step": host_q.numel() * host_q.element_size(),
@@ -658,21 +687,25 @@ def run_reference(args, w, rank, world):
         return None
     inp = make_inputs(w)
     per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
-    vals = []
+    vals, walls = [], []
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         cb = cpu_baseline(w, inp, budget_s=per_step)
         if i >= args.warmup:
             vals.append(cb)
+            walls.append(time.perf_counter() - t0)
     value = statistics.median(c["value"] for c in vals)
-    ms = w.ops / (value * 1e12) * 1e3
     cb = dict(vals[-1])
     cb["value"] = value
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
-                   "bias": w.bias, "parallelism": "cpu oracle"},
+        "steps": args.steps, "warmup": args.warmup,
+        # each step is a bounded sample of the workload: its own wall time,
+        # and the full workload's time at the sample's rate beside it
+        "ms_per_step": statistics.median(walls) * 1e3,
+        "ms_per_step_full_workload_est": w.ops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic", "config": bench_config(w, world, args.variant),
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -683,17 +716,23 @@ def run_reference_decode(args, w, rank, world):
         return None
     inp = make_decode_inputs(w)
     per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
-    vals = [cpu_baseline_decode(w, inp, budget_s=per_step) for _ in range(args.warmup + args.steps)][args.warmup:]
+    vals, walls = [], []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        cb = cpu_baseline_decode(w, inp, budget_s=per_step)
+        if i >= args.warmup:
+            vals.append(cb)
+            walls.append(time.perf_counter() - t0)
     value = statistics.median(c["value"] for c in vals)
     cb = dict(vals[-1])
     cb["value"] = value
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.ops / (value * 1e12) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(walls) * 1e3,
+        "ms_per_step_full_workload_est": w.ops / (value * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
-                   "input_dtype": w.dtype, "bias": "none", "parallelism": "cpu oracle"},
+        "config": decode_config(w, world),
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
