@@ -15,8 +15,9 @@ import ctypes
 
 from . import _native as N
 
-__all__ = ["pack_qk", "quant_v", "attention_fwd", "attention_fwd_noalloc", "attention_workspace",
-           "workspace_bytes", "scores_debug", "forward", "check_device_status", "words", "vq_ld"]
+__all__ = ["pack_qk", "quant_v", "prepass_qkv", "attention_fwd", "attention_fwd_noalloc", "attention_workspace",
+           "workspace_bytes", "attention_bwd", "attention_decode", "scores_debug", "forward",
+           "check_device_status", "words", "vq_ld"]
 
 
 def _torch():
@@ -196,6 +197,40 @@ def attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA
     _call(muq.device, "ba_attention_fwd_noalloc", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld,
           gh, gw, B, H, Nn, d, _p(out), _dt(out), _stream(muq.device))
     return out
+
+
+def attention_bwd(q, k, bq, muq, bk, muk, vq, sv, out, dout, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0,
+                  grid=None, ste_clip=float("inf"), want_dbias=True, workspace=None, grads=None):
+    """Backward of the fused forward with straight-through estimators
+    (ba_attention_bwd): q, k the raw inputs [B,H,N,d] (their |x| decides the
+    clipped estimator), the pre-pass outputs, the forward output `out` and the
+    upstream gradient `dout` (both fp32 [B,H,N,d]).  Returns (dq, dk, dv,
+    dbias) in fp32; dbias is None without a bias or when not wanted.  `grads`
+    may hold preallocated (dq, dk, dv, dbias) tensors."""
+    torch = _torch()
+    _need_cuda(q, k, bq, muq, bk, muk, vq, sv, out, dout)
+    B, H, Nn, d = q.shape
+    dev = q.device
+    kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
+    if grads is not None:
+        dq, dk, dv, dbias = grads
+        if kind == N.BA_BIAS_NONE or not want_dbias:
+            dbias = None
+    else:
+        dq, dk, dv = (torch.empty((B, H, Nn, d), dtype=torch.float32, device=dev) for _ in range(3))
+        dbias = None
+        if want_dbias and kind != N.BA_BIAS_NONE:
+            dbias = torch.empty_like(bias, dtype=torch.float32)
+    if workspace is None:
+        nb = int(N.lib().ba_attention_bwd_workspace_bytes(B, H, Nn))
+        if nb < 0:
+            raise ValueError("invalid sizes for the backward pass")
+        workspace = torch.empty((nb,), dtype=torch.uint8, device=dev)
+    _same_device(q, k, bq, muq, bk, muk, vq, sv, out, dout, bias, workspace)
+    _call(dev, "ba_attention_bwd", _p(q), _p(k), _dt(q), _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind,
+          bp, ld, gh, gw, B, H, Nn, d, _p(out), _p(dout), float(ste_clip), _p(workspace),
+          workspace.numel(), _p(dq), _p(dk), _p(dv), _p(dbias), _stream(dev))
+    return dq, dk, dv, dbias
 
 
 def scores_debug(bq, bk, d, z=None):

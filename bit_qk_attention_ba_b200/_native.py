@@ -36,8 +36,13 @@ SIGNATURES = {
                                       _P, _I, _I, _P]),
     "ba_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I,
                                       _P]),
+    "ba_attention_bwd": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I,
+                              _P, _P, ctypes.c_float, _P, _I64, _P, _P, _P, _P, _P]),
+    "ba_attention_bwd_workspace_bytes": (_I64, [_I, _I, _I]),
     "ba_scores_debug": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "ba_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
+    "ba_test_attention_fwd_starved": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I64, _P, _I, _I, _I64,
+                                           _P]),
     "ba_status_string": (ctypes.c_char_p, [_I]),
 }
 

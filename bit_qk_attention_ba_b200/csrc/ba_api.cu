@@ -33,7 +33,8 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
                            const int8_t* vq, const float* sv, int bias_kind, const float* bias,
                            int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
                            void* workspace, int64_t workspace_bytes,
-                           void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st);
+                           void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st,
+                           int starve_step = -1, uint64_t wait_ns = 2000000000ull);
 bool attn_tc_supports(int bias_kind, int gh, int gw, int N, int d);
 int64_t attn_decode_workspace_bytes(int B, int H, int Nk, int d, int sm_count);
 cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, const uint32_t* bk, const float* muk,
@@ -41,6 +42,12 @@ cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, con
                                int B, int H, int d, void* workspace, void* out, ba_dtype out_dt,
                                cudaStream_t st, int sm_count);
 int64_t attn_tc_workspace_bytes(int B, int H, int N, int d, int bias_kind, int gh, int gw);
+int64_t attn_bwd_workspace_bytes(int B, int H, int N);
+cudaError_t launch_attn_bwd(const void* q, const void* k, ba_dtype dt, const uint32_t* bq, const float* muq,
+                            const uint32_t* bk, const float* muk, const int8_t* vq, const float* sv, int bias_kind,
+                            const float* bias, int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
+                            const float* out, const float* dout, float clip, void* workspace, float* dq, float* dk,
+                            float* dv, float* dbias, cudaStream_t st);
 
 // One status word per device; kernels OR failure bits into it.
 __device__ unsigned g_device_status;
@@ -309,6 +316,58 @@ ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
     if (workspace_bytes < attn_decode_workspace_bytes(B, H, Nk, d, sms)) return BA_ERR_INVALID_ARG;
     return from_cuda(launch_attn_decode(bq, muq, Nq, bk, muk, vq, sv, Nk, bias, bias_ld, B, H, d, workspace, out,
                                         out_dt, static_cast<cudaStream_t>(stream), sms));
+}
+
+int64_t ba_attention_bwd_workspace_bytes(int B, int H, int N)
+{
+    if (!sizes_ok(B, H, N, 1)) return -1;
+    return attn_bwd_workspace_bytes(B, H, N);
+}
+
+ba_status ba_attention_bwd(const void* q, const void* k, ba_dtype dt,
+                           const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv,
+                           int bias_kind, const float* bias, int64_t bias_ld, int grid_h, int grid_w,
+                           int B, int H, int N, int d,
+                           const float* out, const float* dout, float ste_clip,
+                           void* workspace, int64_t workspace_bytes,
+                           float* dq, float* dk, float* dv, float* dbias, void* stream)
+{
+    if (!sizes_ok(B, H, N, d) || (dt != BA_F32 && dt != BA_BF16)) return BA_ERR_INVALID_ARG;
+    if (!ptr_ok(q, esize(dt)) || !ptr_ok(k, esize(dt)) || !ptr_ok(bq, 4) || !ptr_ok(muq, 4) || !ptr_ok(bk, 4) ||
+        !ptr_ok(muk, 4) || !ptr_ok(vq, 1) || !ptr_ok(sv, 4) || !ptr_ok(out, 4) || !ptr_ok(dout, 4) ||
+        !ptr_ok(dq, 4) || !ptr_ok(dk, 4) || !ptr_ok(dv, 4) || (dbias != nullptr && !ptr_ok(dbias, 4)))
+        return BA_ERR_INVALID_ARG;
+    if (bias_kind == BA_BIAS_DENSE ? !(ptr_ok(bias, 4) && bias_ld >= N) : !bias_ok(bias_kind, bias, bias_ld, grid_h, grid_w, N))
+        return BA_ERR_INVALID_ARG;
+    if (!(ste_clip >= 0.f)) return BA_ERR_INVALID_ARG;            // NaN or negative
+    if (!ptr_ok(workspace, 256) || workspace_bytes < attn_bwd_workspace_bytes(B, H, N)) return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
+    return from_cuda(launch_attn_bwd(q, k, dt, bq, muq, bk, muk, vq, sv, bias_kind, bias, bias_ld, grid_h, grid_w,
+                                     B, H, N, d, out, dout, ste_clip, workspace, dq, dk, dv, dbias,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+ba_status ba_test_attention_fwd_starved(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                                        const int8_t* vq, const float* sv, int B, int H, int N, int d,
+                                        void* workspace, int64_t workspace_bytes, void* out, ba_dtype out_dt,
+                                        int starve_step, int64_t wait_ns, void* stream)
+{
+    const ba_status v = validate_fwd(bq, muq, bk, muk, vq, sv, BA_BIAS_NONE, nullptr, 0, 0, 0, B, H, N, d, out,
+                                     out_dt);
+    if (v != BA_OK) return v;
+    if (starve_step < 0 || wait_ns < 1000000 || wait_ns > 2000000000ll) return BA_ERR_INVALID_ARG;
+    if (!attn_tc_supports(BA_BIAS_NONE, 0, 0, N, d)) return BA_ERR_UNSUPPORTED;
+    if (!ptr_ok(workspace, 256) || workspace_bytes < attn_tc_workspace_bytes(B, H, N, d, BA_BIAS_NONE, 0, 0))
+        return BA_ERR_INVALID_ARG;
+    if (const ba_status e = check_stream(stream)) return e;
+    unsigned* status = device_status_ptr();
+    if (!status) return BA_ERR_CUDA;
+    const cudaError_t e = launch_attn_tc(bq, muq, bk, muk, vq, sv, BA_BIAS_NONE, nullptr, 0, 0, 0, B, H, N, d,
+                                         workspace, workspace_bytes, out, out_dt, BA_QK_AUTO, status,
+                                         static_cast<cudaStream_t>(stream), starve_step, (uint64_t)wait_ns);
+    if (e == cudaErrorNotSupported) return BA_ERR_UNSUPPORTED;
+    return from_cuda(e);
 }
 
 ba_status ba_check_device_status(void* stream, int* code)

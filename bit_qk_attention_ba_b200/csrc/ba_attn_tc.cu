@@ -13,9 +13,11 @@
 // Blackwell:
 //   * a CTA owns 128 query rows (row = TMEM lane) and walks the keys in
 //     steps of 128: one QK product of N = 128 per step, the widest tile whose
-//     S fits three times in TMEM next to the output accumulator.  Two softmax
-//     threads share a row, each taking 64 keys of a step; they combine their
-//     row maxima once (end of pass A) and their row sums once (epilogue);
+//     S fits three times in TMEM next to the output accumulator.  Four softmax
+//     threads share a row, each taking 32 keys of a step (16 softmax warps, so
+//     four per SM sub-partition hide each other's TMEM-load and arithmetic
+//     latency); they combine their row maxima once (end of pass A) and their
+//     row sums once (epilogue);
 //   * the keys are swept twice: pass A finds the exact row maximum m_i, pass
 //     B quantises P~ = exp(S - m_i) against it.  The u8 codes are then the
 //     ones an exact-maximum reference produces, and the int32 PV accumulator
@@ -35,14 +37,14 @@
 //   * PV runs on tcgen05.mma kind::i8 with u8 P read straight from TMEM (each
 //     softmax thread writes its codes over the S columns it has already read)
 //     and s8 V tiles, accumulating in TMEM across all key tiles;
-//   * the softmax pulls its 64 keys of an S tile out of TMEM with one load
+//   * the softmax pulls its 32 keys of an S tile out of TMEM with one load
 //     and does its arithmetic on packed fp32 pairs (fma/mul/add .f32x2) with
 //     a 3-input max; a bias window is read as reversed copies, four keys per
 //     16-byte load;
 //   * ring slots and mbarrier parities are counters advanced once per step
 //     (no division by the runtime stage count).
-// Warps 0-7 run the softmax (warp w: TMEM lanes 32 (w % 4) .., keys
-// 64 (w / 4) .. of each step), warp 8 loads, warp 9 issues the MMAs and owns
+// Warps 0-15 run the softmax (warp w: TMEM lanes 32 (w % 4) .., keys
+// 32 (w / 4) .. of each step), warp 16 loads, warp 17 issues the MMAs and owns
 // TMEM.
 //
 // Every wait on an mbarrier is bounded; on a timeout the kernel records a bit
@@ -61,15 +63,17 @@ namespace tc {
 namespace {
 
 constexpr int BN = 128;                 // keys per step (N of the QK product)
-constexpr int HALVES = 2;               // softmax threads per row
-constexpr int KH = BN / HALVES;         // keys per softmax thread per step
+constexpr int KQ = 4;                   // softmax threads per row (key quarters of a step)
+constexpr int KT = BN / KQ;             // keys per softmax thread per step (32)
 constexpr int NSB = 3;                  // S buffers in TMEM
 constexpr uint32_t O_COL = NSB * BN;    // TMEM column of the output accumulator
 constexpr int MAX_STAGES = 4;
-constexpr int NUM_SOFTMAX_WARPS = 4 * HALVES;               // 8
-constexpr int LOAD_WARP = NUM_SOFTMAX_WARPS;                // 8
-constexpr int MMA_WARP = LOAD_WARP + 1;                     // 9
-constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 320
+constexpr int NUM_SOFTMAX_WARPS = 4 * KQ;                   // 16
+constexpr int LOAD_WARP = NUM_SOFTMAX_WARPS;                // 16
+constexpr int MMA_WARP = LOAD_WARP + 1;                     // 17
+constexpr int NUM_THREADS = 32 * (MMA_WARP + 1);            // 576
+// 576 threads share the 64K-entry register file: at most 113 registers each
+// (the launch bound below lets the compiler know).
 constexpr int RP_WIN = 256;             // entries per shifted copy of a window (255 used)
 constexpr int RP_STRIDE = 264;          // floats between copies in shared memory (8 words mod 32)
 constexpr uint32_t RP_COPY_BYTES = RP_WIN * 4;
@@ -95,7 +99,7 @@ struct Layout {
     uint32_t q, q_bytes;        // Q operand
     uint32_t k, k_bytes;        // [stage] staged key tile
     uint32_t rp;                // [stage][4][RP_STRIDE] rel-pos window copies
-    uint32_t xmax, xsum;        // [HALVES][BM] partial row maxima / sums
+    uint32_t xmax, xsum;        // [KQ][BM] partial row maxima / sums
     uint32_t bars, misc, total;
 };
 
@@ -113,8 +117,8 @@ __host__ __device__ inline Layout make_layout(int dpad, int dv, int bias_kind, i
     L.k_bytes = align_up(L.tile, 128);
     L.k = off; off += stages * L.k_bytes;
     L.rp = off; off += (bias_kind == BIAS_RP_FAST) ? stages * 4 * RP_STRIDE * 4u : 0u;
-    L.xmax = off; off += HALVES * BM * 4;
-    L.xsum = off; off += HALVES * BM * 4;
+    L.xmax = off; off += KQ * BM * 4;
+    L.xsum = off; off += KQ * BM * 4;
     L.bars = off; off += NUM_BARS * 8;
     L.misc = off; off += 16;            // TMEM base address, abort flag
     L.total = off;
@@ -133,10 +137,12 @@ struct Params {
     int gh, gw;
     float q_scale;           // 1 / sqrt(d)
     unsigned* status;
+    uint64_t wait_ns;        // give-up time of every barrier wait (2 s in production)
+    int starve_step;         // testing only: the loader stops before this step (-1: never)
 };
 
 template <int QK, typename OutT, int BIAS>
-__global__ void __maxnreg__(MAX_REGS)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
                const Params p)
 {
@@ -214,7 +220,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 const bool pass_b = u >= T;
                 const int t = pass_b ? u - T : u;
                 const int j0 = t * BN;
-                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag)) {
+                // Testing only: issue nothing from this step on, so the roles
+                // that wait for it give up (no copy is left in flight: the MMA
+                // warp has waited for every earlier stage before it reaches
+                // this one).
+                if (u == p.starve_step) break;
+                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag, p.wait_ns)) {
                     fail(abort_flag, p.status, kStatusTimeoutProducer);
                     break;
                 }
@@ -254,7 +265,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                                                     : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
             const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
             const uint32_t sbo_qk = (uint32_t)chunks * 128u;
-            bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag);
+            bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag, p.wait_ns);
             // Descriptors are built once; moving along a buffer only adds to the
             // start-address field (bytes / 16), which never carries out.
             const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
@@ -272,8 +283,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             uint32_t q_sp = 0, q_bp = 0;
             auto issue_qk = [&](int u) -> bool {
                 const int s = q_s, b = q_b;
-                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
-                if (u >= NSB && !mbar_wait(&bars[B_SDONE + b], q_bp ^ 1u, abort_flag)) return false;
+                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag, p.wait_ns)) return false;
+                if (u >= NSB && !mbar_wait(&bars[B_SDONE + b], q_bp ^ 1u, abort_flag, p.wait_ns)) return false;
                 tc_fence_after();
                 const uint64_t dk = dk0 + s * k_step;
                 const uint32_t d_tmem = tmem + b * BN;
@@ -294,14 +305,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 if (u + LA < U && !(ok = issue_qk(u + LA))) break;
                 if (u >= T) {
                     // PV: u8 P x s8 V, K = 32 keys per product.  The P codes of
-                    // keys 64 h .. 64 h + 63 sit in columns 64 h .. 64 h + 15 of
-                    // the S buffer.
+                    // keys 32 kq .. 32 kq + 31 sit in columns 32 kq .. 32 kq + 7
+                    // of the S buffer.
                     const int t = u - T, b = p_b, s = p_s;
-                    if (!(ok = mbar_wait(&bars[B_SDONE + b], p_bp, abort_flag))) break;
+                    if (!(ok = mbar_wait(&bars[B_SDONE + b], p_bp, abort_flag, p.wait_ns))) break;
                     tc_fence_after();
                     const uint32_t a_tmem = tmem + b * BN;
                     for (int kk = 0; kk < BN / 32; ++kk)
-                        mma_ts_i8(tmem + O_COL, a_tmem + (kk >> 1) * KH + (kk & 1) * 8,
+                        mma_ts_i8(tmem + O_COL, a_tmem + kk * KT,
                                   dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
                                   idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -317,18 +328,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
         const int quarter = warp & 3;                 // TMEM lanes this warp may access
-        const int hf = warp >> 2;                     // which 64 keys of each step
+        const int kq = warp >> 2;                     // which 32 keys of each step
         const int r = quarter * 32 + lane;            // row within the CTA
         const int i = q0 + r;
         const bool row_ok = i < N;
         const int ie = row_ok ? i : N - 1;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
-        // Q operand of this row, padding channels zeroed (the halves split the words).
+        // Q operand of this row, padding channels zeroed (the row's threads split the words).
         {
             uint8_t* qop = smem + L.q;
             const uint32_t* src = p.bq + ((size_t)bh * N + ie) * W;
-            for (int w = hf; w < W; w += HALVES) {
+            for (int w = kq; w < W; w += KQ) {
                 const uint32_t bits = row_ok ? __ldg(src + w) : 0u;
                 const int nvalid = min(32, p.d - 32 * w);
                 const uint32_t vm = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
@@ -349,7 +360,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 // starts that run on a 16-byte boundary.
                 const int sidx = (BM - 1) - r;
                 const int m = sidx & 3;
-                rp_off = m * RP_STRIDE + (sidx - m) + hf * KH;
+                rp_off = m * RP_STRIDE + (sidx - m) + kq * KT;
             } else {
                 // Patch index of the row; the class row (token 0 with a class
                 // token) gathers from the table centre, always in range, and
@@ -371,45 +382,45 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
             const int s = r_s, b = r_b;
             const bool pass_b = u >= T;
             const int t = pass_b ? u - T : u;
-            const int jh = t * BN + hf * KH;          // first key of this thread's half
-            ok = warp_wait(&bars[B_SFULL + b], r_bp, abort_flag) &&
-                 warp_wait(&bars[B_FULL + s], r_sp, abort_flag);
+            const int jh = t * BN + kq * KT;          // first key of this thread's quarter
+            ok = warp_wait(&bars[B_SFULL + b], r_bp, abort_flag, p.wait_ns) &&
+                 warp_wait(&bars[B_FULL + s], r_sp, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
-            const bool ragged = jh + KH > N;
+            const bool ragged = jh + KT > N;
             const uint8_t* tile_s = smem + L.k + s * L.k_bytes;
-            const float* muk_s = reinterpret_cast<const float*>(tile_s + BN * p.dpad) + hf * KH;
-            const int* koff_s = reinterpret_cast<const int*>(tile_s + BN * p.dpad + BN * 4) + hf * KH;
-            const uint8_t* bsm_row = smem + L.b + (s * 4 + 2 * hf) * 16384 + r * 128;
+            const float* muk_s = reinterpret_cast<const float*>(tile_s + BN * p.dpad) + kq * KT;
+            const int* koff_s = reinterpret_cast<const int*>(tile_s + BN * p.dpad + BN * 4) + kq * KT;
+            const uint8_t* bsm_row = smem + L.b + (s * 4 + kq) * 16384 + r * 128;
             const float* rpc = (BIAS == BIAS_RP_FAST)
                 ? reinterpret_cast<const float*>(smem + L.rp) + (size_t)s * 4 * RP_STRIDE + rp_off : nullptr;
             const int nvalid = N - jh;
             const uint32_t s_col = tmem + b * BN;
-            uint32_t zr[64];
-            tmem_ld64(s_col + hf * KH + lane_base, zr);
+            uint32_t zr[KT];
+            tmem_ld32(s_col + kq * KT + lane_base, zr);
             tmem_wait_ld();
-            uint32_t pw[16];
+            uint32_t pw[KT / 4];
             float mx[2] = {-INFINITY, -INFINITY};
             if (!pass_b) {
                 if (ragged)
-                    softmax_tile<QK, BIAS, false, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                    softmax_tile<QK, BIAS, false, true, KT>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                         nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 else
-                    softmax_tile<QK, BIAS, false, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                    softmax_tile<QK, BIAS, false, false, KT>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                          nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 mrow = fmax3(mrow, mx[0], mx[1]);
             } else {
                 if (ragged)
-                    softmax_tile<QK, BIAS, true, true>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                    softmax_tile<QK, BIAS, true, true, KT>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                        nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
                 else
-                    softmax_tile<QK, BIAS, true, false>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
+                    softmax_tile<QK, BIAS, true, false, KT>(zr, muk_s, bsm_row, r & 7, rpc, koff_s, tab_h, rel_base,
                                                         nvalid, cq2, neg2, mx, l2, pw, cls3, cls_row);
-                // The u8 codes of these 64 keys go back into this row's lane of
-                // the S buffer, over the first 16 columns of this thread's own
-                // half (already read; the other half's S columns are never
-                // written here): the PV product reads them from TMEM.
-                tmem_st16(s_col + hf * KH + lane_base, pw);
+                // The u8 codes of these 32 keys go back into this row's lane of
+                // the S buffer, over the first 8 columns of this thread's own
+                // quarter (already read; the other quarters' S columns are
+                // never written here): the PV product reads them from TMEM.
+                tmem_st8(s_col + kq * KT + lane_base, pw);
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -419,38 +430,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 mbar_arrive(&bars[B_EMPTY + s]);
             }
             if (u == T - 1) {
-                // Row maximum = the larger of the two halves' maxima.
+                // Row maximum = the largest of the quarters' maxima.
                 float* xm = reinterpret_cast<float*>(smem + L.xmax);
-                xm[hf * BM + r] = mrow;
+                xm[kq * BM + r] = mrow;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_XMAX]);
-                if (!warp_wait(&bars[B_XMAX], 0, abort_flag)) { ok = false; break; }
-                mrow = fmaxf(xm[r], xm[BM + r]);
+                if (!warp_wait(&bars[B_XMAX], 0, abort_flag, p.wait_ns)) { ok = false; break; }
+                mrow = fmaxf(fmax3(xm[r], xm[BM + r], xm[2 * BM + r]), xm[3 * BM + r]);
                 neg2 = f2_pack(-mrow * LOG2E, -mrow * LOG2E);
             }
         }
 
-        // Epilogue: O = sv * acc / (255 l), l = the two halves' sums in a fixed order.
-        if (ok) ok = warp_wait(&bars[B_OREADY], 0, abort_flag);
+        // Epilogue: O = sv * acc / (255 l), l = the quarters' sums in a fixed order.
+        if (ok) ok = warp_wait(&bars[B_OREADY], 0, abort_flag, p.wait_ns);
         if (ok) {
             float la, lb, lc, ld;
             f2_unpack(l2[0], la, lb);
             f2_unpack(l2[1], lc, ld);
             float* xs = reinterpret_cast<float*>(smem + L.xsum);
-            xs[hf * BM + r] = (la + lb) + (lc + ld);
+            xs[kq * BM + r] = (la + lb) + (lc + ld);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_XSUM]);
-            ok = warp_wait(&bars[B_XSUM], 0, abort_flag);
+            ok = warp_wait(&bars[B_XSUM], 0, abort_flag, p.wait_ns);
         }
         if (!ok) {
             if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutSoftmax);
         } else {
             tc_fence_after();
             const float* xs = reinterpret_cast<const float*>(smem + L.xsum);
-            const float inv = 1.f / (255.f * (xs[r] + xs[BM + r]));
+            const float inv = 1.f / (255.f * ((xs[r] + xs[BM + r]) + (xs[2 * BM + r] + xs[3 * BM + r])));
             OutT* dst = static_cast<OutT*>(p.out) + ((size_t)bh * N + ie) * p.d;
             const float* svp = p.sv + (size_t)bh * p.d;
-            for (int c = hf * 16; c < p.dv; c += 16 * HALVES) {
+            for (int c = kq * 16; c < p.dv; c += 16 * KQ) {
                 uint32_t acc[16];
                 tmem_ld16(tmem + O_COL + c + lane_base, acc);
                 tmem_wait_ld();
@@ -611,9 +622,12 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
                            const int8_t* vq, const float* sv, int bias_kind, const float* bias,
                            int64_t bias_ld, int gh, int gw, int B, int H, int N, int d,
                            void* workspace, int64_t workspace_bytes,
-                           void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st)
+                           void* out, ba_dtype out_dt, int variant, unsigned* status, cudaStream_t st,
+                           int starve_step, uint64_t wait_ns)
 {
     if (!attn_tc_supports(bias_kind, gh, gw, N, d)) return cudaErrorNotSupported;
+    // the starved-loader test mode exists for the 128-key kernel only
+    if (starve_step >= 0 && use_pair(bias_kind, B)) return cudaErrorNotSupported;
     const Workspace ws = workspace_layout(B, H, N, d, bias_kind, gh, gw);
     if (workspace == nullptr || workspace_bytes < ws.total) return cudaErrorInvalidValue;
     auto encode = encode_fn();
@@ -662,6 +676,8 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     p.gh = gh; p.gw = gw;
     p.q_scale = (float)(1.0 / sqrt((double)d));
     p.status = status;
+    p.wait_ns = wait_ns;
+    p.starve_step = starve_step;
 
     // Staging pre-passes (same stream, so the attention kernel sees them).
     {

@@ -90,9 +90,10 @@ __device__ __forceinline__ uint32_t core_off(int r, int kc, int chunks)
 }
 
 // Warp-uniform bounded wait: every lane polls, all agree on the outcome.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = 2000000000ull)
 {
-    const bool ok = mbar_wait(bar, parity, abort_flag);
+    const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -148,19 +149,20 @@ __device__ __forceinline__ void store_out16(OutT* dst, const uint32_t (&acc)[16]
     }
 }
 
-// 64 keys of one row: S = z * mu_k * cq + b (Key design 2) on packed
-// pairs, then either the row maximum (pass A) or P~ = exp(S - m), the row sum
-// and the u8 codes round(255 P~) (pass B).  MASK drops keys >= N.  Two
-// independent max / sum accumulators keep the dependency chains short.
+// KEYS (64 or 32) keys of one row: S = z * mu_k * cq + b (Key design 2) on
+// packed pairs, then either the row maximum (pass A) or P~ = exp(S - m), the
+// row sum and the u8 codes round(255 P~) (pass B).  MASK drops keys >= N.
+// Two independent max / sum accumulators keep the dependency chains short.
 // For BIAS_RP_CLS, cls3 points at the head's three class entries (class
 // query -> patch key, patch query -> class key, class -> class), a key offset
 // of -1 marks the class key, and cls_row marks the class query's row.
-template <int QK, int BIAS, bool PASS_B, bool MASK>
-__device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const float* mks, const uint8_t* bsm_row,
+template <int QK, int BIAS, bool PASS_B, bool MASK, int KEYS = TILE_KEYS, bool EXP16 = false>
+__device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[KEYS], const float* mks, const uint8_t* bsm_row,
                                              int bsm_sw, const float* rp_copy, const int* koff,
                                              const float* tab_h, int rel_base, int nvalid,
                                              uint64_t cq2, uint64_t neg2, float (&mx)[2], uint64_t (&l2)[2],
-                                             uint32_t (&pw)[16], const float* cls3 = nullptr, bool cls_row = false)
+                                             uint32_t (&pw)[KEYS / 4], const float* cls3 = nullptr,
+                                             bool cls_row = false)
 {
     float c2t = 0.f, key_cls = 0.f;
     if (BIAS == BIAS_RP_CLS) {
@@ -196,10 +198,10 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
 #pragma unroll
     for (int k = 0; k < PF; ++k) fetch(k, mkq[k], bbq[k]);
 #pragma unroll
-    for (int k4 = 0; k4 < TILE_KEYS / 4; ++k4) {
+    for (int k4 = 0; k4 < KEYS / 4; ++k4) {
         const float4 mk = mkq[k4 % PF];
         const float4 bb = bbq[k4 % PF];
-        if (k4 + PF < TILE_KEYS / 4) fetch(k4 + PF, mkq[k4 % PF], bbq[k4 % PF]);
+        if (k4 + PF < KEYS / 4) fetch(k4 + PF, mkq[k4 % PF], bbq[k4 % PF]);
         uint64_t z01, z23;
         if (QK == QK_F8) {
             z01 = f2_pack(__uint_as_float(zr[4 * k4]), __uint_as_float(zr[4 * k4 + 1]));
@@ -231,6 +233,18 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&zr)[64], const flo
             f2_unpack(s23, c, e);
             mx[k4 & 1] = fmax3(mx[k4 & 1], a, b);
             mx[k4 & 1] = fmax3(mx[k4 & 1], c, e);
+        } else if (EXP16) {
+            // P~ on the f16x2 path: one MUFU operation gives two exponentials;
+            // the codes come from an f16 fma (255 P~ + 1024 has ulp 1, so its
+            // low byte is round-half-even(255 P~)); the row sum stays fp32.
+            float a, b, c, e;
+            f2_unpack(f2_fma(s01, L2E, neg2), a, b);
+            f2_unpack(f2_fma(s23, L2E, neg2), c, e);
+            const uint32_t h01 = ex2_f16x2(f16x2_from(a, b));
+            const uint32_t h23 = ex2_f16x2(f16x2_from(c, e));
+            constexpr uint32_t H255 = 0x5BF85BF8u, H1024 = 0x64006400u;
+            pw[k4] = __byte_perm(fma_f16x2(h01, H255, H1024), fma_f16x2(h23, H255, H1024), 0x6420);
+            l2[k4 & 1] = f2_add(l2[k4 & 1], f2_add(f2_from_f16x2(h01), f2_from_f16x2(h23)));
         } else {
             float a, b, c, e;
             f2_unpack(f2_fma(s01, L2E, neg2), a, b);

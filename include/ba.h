@@ -227,6 +227,44 @@ ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
 int64_t ba_attention_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
 /*
+ * KD4 -- the training-side backward pass (quantisation-aware training with a
+ * straight-through estimator for sign; the page's "QAT + Self-Distillation"
+ * key design and its "Loss and training strategy" paragraph).  Readings: every
+ * quantiser -- sign, the u8 rounding of P~, the int8 rounding of V -- passes
+ * its gradient straight through, the sign's only where |x| <= ste_clip
+ * (INFINITY for the plain identity estimator); the scale mu = mean |x|, the
+ * bias and the softmax are differentiated exactly; the row maximum is a
+ * constant.  With P = P~ / l, P^ = round(255 P~) / (255 l), V^ = sv vq:
+ *   dv_j  = sum_i P^_ij dO_i
+ *   dS_ij = P_ij (dO_i . V^_j - dO_i . O_i)
+ *   dq_ic = [|q_ic| <= ste_clip] sum_j dS_ij mu_q,i mu_k,j t_jc / sqrt(d)
+ *           + sign(q_ic) / d * sum_j dS_ij mu_k,j z_ij / sqrt(d)      (dk likewise)
+ *   dbias = dS summed over the batch and over every (i, j) reading an entry.
+ * Inputs: q, k [B, H, N, d] raw values (dtype dt; only their signs, already in
+ *   bq / bk, and |x| <= ste_clip are used); bq, muq, bk, muk, vq, sv as for
+ *   ba_attention_fwd; the bias arguments as there; out: the forward output O
+ *   [B, H, N, d] fp32; dout: dO [B, H, N, d] fp32.
+ * Outputs (fp32): dq, dk, dv [B, H, N, d]; dbias (NULL to skip) in the bias's
+ *   own shape (dense [H, N, bias_ld], columns >= N set to 0; table [H, G] or
+ *   [H, G + 3]), overwritten.  The bias gradient is summed with atomics, so
+ *   its last bits depend on the order of the additions.
+ * workspace: at least ba_attention_bwd_workspace_bytes(B, H, N) bytes of
+ *   device scratch, 256-byte aligned, owned by the caller (row statistics).
+ * Runs on CUDA cores (four launches: row statistics, dq with dbias, dk, dv).
+ */
+ba_status ba_attention_bwd(const void* q, const void* k, ba_dtype dt,
+                           const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                           const int8_t* vq, const float* sv,
+                           int bias_kind, const float* bias, int64_t bias_ld, int grid_h, int grid_w,
+                           int B, int H, int N, int d,
+                           const float* out, const float* dout, float ste_clip,
+                           void* workspace, int64_t workspace_bytes,
+                           float* dq, float* dk, float* dv, float* dbias, void* stream);
+
+/* Workspace bytes ba_attention_bwd needs; -1 for invalid sizes. */
+int64_t ba_attention_bwd_workspace_bytes(int B, int H, int N);
+
+/*
  * KD1 -- the integer binary score matrix, for checking and debugging.
  *   z : [B, H, N, N] int32, z[b][h][i][j] = d - 2 popcount(bq_i XOR bk_j).
  */
@@ -239,6 +277,23 @@ ba_status ba_scores_debug(const uint32_t* bq, const uint32_t* bk,
  * BA_ERR_DEVICE_STATUS with the recorded bits in *code (may be NULL).
  */
 ba_status ba_check_device_status(void* stream, int* code);
+
+/*
+ * TESTING ONLY -- exercises the bounded waits of the tensor-core forward.
+ * Runs ba_attention_fwd (no bias, the 128-key tensor-core kernel) with its
+ * loader stopping before key step `starve_step` (0-based over both sweeps)
+ * and every barrier wait giving up after `wait_ns` nanoseconds (1 ms .. 2 s).
+ * Every copy issued before that step has been consumed when the waits give
+ * up, so nothing is left in flight: the roles record their bits in the
+ * device status word, release tensor memory and return; out is undefined.
+ * ba_check_device_status then reports BA_ERR_DEVICE_STATUS, and the next
+ * normal call runs clean.  BA_ERR_UNSUPPORTED for shapes that do not run
+ * the 128-key kernel.  Not part of the method: no production path calls it.
+ */
+ba_status ba_test_attention_fwd_starved(const uint32_t* bq, const float* muq, const uint32_t* bk, const float* muk,
+                                        const int8_t* vq, const float* sv, int B, int H, int N, int d,
+                                        void* workspace, int64_t workspace_bytes, void* out, ba_dtype out_dt,
+                                        int starve_step, int64_t wait_ns, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* ba_status_string(ba_status s);
