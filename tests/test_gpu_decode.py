@@ -15,6 +15,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 import bit_qk_attention_ba_b200 as ba  # noqa: E402
+from guard import Guarded  # noqa: E402
 from bit_qk_attention_ba_b200 import _native as NAT  # noqa: E402
 
 DEV = torch.device("cuda:0")
@@ -42,8 +43,12 @@ def _run(q, k, v, b, d):
     bk, muk = ba.pack_qk(k.to(DEV))
     vq, sv = ba.quant_v(v.to(DEV))
     bt = None if b is None else torch.from_numpy(b).to(DEV)
-    out = ba.attention_decode(bq, muq, bk, muk, vq, sv, d, bias=bt)
+    guard = Guarded()
+    B, H, Nq = muq.shape
+    out = ba.attention_decode(bq, muq, bk, muk, vq, sv, d, bias=bt,
+                              out=guard.empty((B, H, Nq, d), torch.float32, DEV))
     torch.cuda.synchronize()
+    guard.check()
     return out.cpu().numpy()
 
 

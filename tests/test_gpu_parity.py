@@ -24,6 +24,7 @@ if not torch.cuda.is_available():
 
 import bit_qk_attention_ba_b200 as ba  # noqa: E402
 from bit_qk_attention_ba_b200 import _native as NAT  # noqa: E402
+from guard import Guarded  # noqa: E402
 
 DEV = torch.device("cuda:0")
 MAX_ABS, MEAN_ABS = 2e-2, 2e-3
@@ -66,13 +67,20 @@ def _bias_gpu(inp, w):
 
 
 def _run_gpu(w, inp, variant=NAT.BA_QK_AUTO, out_dtype=torch.float32):
-    """The benchmarked hot path: the fused pre-pass, then the attention call."""
+    """The benchmarked hot path: the fused pre-pass, then the attention call.
+    Every output sits inside guard bytes, checked after the kernels ran."""
     q, k, v = (_gpu(inp[n], w.dtype) for n in ("q", "k", "v"))
-    bq, muq, bk, muk, vq, sv = ba.prepass_qkv(q, k, v)
+    g = Guarded()
+    B, H, N, d = w.B, w.H, w.N, w.d
+    outs = (g.empty((B, H, N, ba.words(d)), torch.int32, DEV), g.empty((B, H, N), torch.float32, DEV),
+            g.empty((B, H, N, ba.words(d)), torch.int32, DEV), g.empty((B, H, N), torch.float32, DEV),
+            g.empty((B, H, d, ba.vq_ld(N)), torch.int8, DEV), g.empty((B, H, d), torch.float32, DEV))
+    bq, muq, bk, muk, vq, sv = ba.prepass_qkv(q, k, v, outs)
     out = ba.attention_fwd(bq, muq, bk, muk, vq, sv, w.d, bias=_bias_gpu(inp, w),
                            bias_kind=BIAS_KIND[w.bias], ld=inp["ld"], grid=w.grid,
-                           out_dtype=out_dtype, variant=variant)
+                           out=g.empty((B, H, N, d), out_dtype, DEV), variant=variant)
     torch.cuda.synchronize()
+    g.check()
     return dict(bq=bq, muq=muq, bk=bk, muk=muk, vq=vq, sv=sv, out=out)
 
 
