@@ -323,6 +323,47 @@ def time_side_workload(w, variant, dev, steps=50, warmup=10):
             "roofline": roof, "device_status": status}
 
 
+def time_backward(w, dev, steps=10, warmup=3):
+    """The training-side backward (ba_attention_bwd: straight-through
+    estimators, CUDA cores) on workload w: CUDA events around the call,
+    median over the timed steps.  Ops counted: the four N x N x d
+    contractions of an attention backward (dO V^T, P^T dO, dS K, dS^T Q),
+    8 B H N^2 d; roofline: fp32 FMA on the CUDA cores (148 SMs x 128 lanes x
+    2 flop x the SM clock)."""
+    import torch
+    import bit_qk_attention_ba_b200 as ba
+    inp = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v = (torch.from_numpy(inp[n]).to(tdt).to(dev) for n in ("q", "k", "v"))
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
+    kind, ld, grid = BIAS_KIND[w.bias], inp["ld"], w.grid
+    pre = ba.prepass_qkv(q, k, v)
+    out = ba.attention_fwd(*pre, w.d, bias=bias, bias_kind=kind, ld=ld, grid=grid, out_dtype=torch.float32)
+    dout = torch.randn(out.shape, generator=torch.Generator(device="cpu").manual_seed(0)).to(dev)
+    grads = None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warmup + steps):
+        e = ev[i - warmup] if i >= warmup else None
+        if e:
+            e[0].record(stream)
+        grads = ba.attention_bwd(q, k, *pre, out, dout, bias=bias, bias_kind=kind, ld=ld, grid=grid, grads=grads)
+        if e:
+            e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    ops = 8.0 * w.B * w.H * w.N * w.N * w.d
+    peak = 148 * 128 * 2 * 1965e6 / 1e12
+    status = ba.check_device_status(dev)
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": w.bias, "ms": ms,
+            "tops": ops / (ms * 1e-3) / 1e12, "launches": 4,
+            "roofline": {"bound": "alu", "achieved": ops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": ops / (ms * 1e-3) / 1e12 / peak,
+                         "peak_source": "fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x 1965 MHz",
+                         "ops": ops},
+            "device_status": status}
+
+
 def run_ours(args, w, rank, local_rank, world):
     import torch
     import bit_qk_attention_ba_b200 as ba
@@ -480,6 +521,8 @@ def run_ours(args, w, rank, local_rank, world):
         "clocks": clocks,
         "device_status": status,
     }
+    if not args.no_backward:
+        line["backward"] = time_backward(WORKLOADS["deit_b384"], dev)
     if not args.no_side_workloads:
         # every rank times the same side workloads, so the ranks stay in step
         side = {}
@@ -748,6 +791,7 @@ def main(argv=None):
     ap.add_argument("--variant", type=int, default=0, help="QK path: 0 auto, 1 popc, 2 mma.sync b1, 3 tcgen05 i8, 4 tcgen05 f8")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training-side backward timing")
     ap.add_argument("--no-side-workloads", action="store_true",
                     help="skip the gate workloads timed beside the headline one")
     args = ap.parse_args(argv)
