@@ -41,8 +41,19 @@ from bit_qk_attention_ba_b200.workloads import (BIAS_KIND, DECODE_WORKLOADS, WOR
                                                 make_decode_inputs, make_inputs)
 
 METRIC = "binary attention effective TOPS (4*B*H*N^2*d per step)"
-DTYPE = ("+-1 int8 QK on tcgen05 kind::i8 (s32 accumulate), u8 x s8 PV on tcgen05 kind::i8 (s32), "
-         "fp32 scores and softmax")
+def dtype_of(w, variant):
+    """The arithmetic the attention path runs for workload w: the QK kind the
+    library picks (kind::f8f6f4 with +-1 e4m3 operands in the 128-key kernel,
+    kind::i8 in the paired one, unless a variant is forced)."""
+    pv = "u8 x s8 PV on tcgen05 kind::i8 (s32), fp32 scores and softmax"
+    if variant == 1:
+        return "b1 QK by XOR/popcount on CUDA cores, u8 x s8 PV by dp4a (s32), fp32 softmax"
+    if variant == 2:
+        return "b1 QK on warp mma.sync .b1 xor.popc, u8 x s8 PV on mma.sync (s32), fp32 softmax"
+    f8 = variant == 4 or (variant == 0 and attn_kernel(w, variant)[0] == "attn_tc_kernel")
+    if f8:
+        return "+-1 e4m3 QK on tcgen05 kind::f8f6f4 (fp32 accumulate, exact), " + pv
+    return "+-1 int8 QK on tcgen05 kind::i8 (s32 accumulate), " + pv
 # The gate workloads reported beside the headline one, each timed on its own.
 SIDE_WORKLOADS = ("deit_b384", "deit_s", "dit_xl2", "deit_t")
 L2_BYTES = 126 * 2 ** 20
@@ -511,7 +522,7 @@ def run_ours(args, w, rank, local_rank, world):
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype_of(w, args.variant), "data": "synthetic",
         "config": bench_config(w, world, args.variant),
         "roofline": roof,
         "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
@@ -792,6 +803,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the training-side backward timing")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller cases for profiler captures)")
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiler captures)")
     ap.add_argument("--no-side-workloads", action="store_true",
                     help="skip the gate workloads timed beside the headline one")
     args = ap.parse_args(argv)
@@ -808,6 +822,8 @@ def main(argv=None):
             print(json.dumps(line), flush=True)
         return
     w = WORKLOADS[args.workload]
+    if args.batch or args.heads:
+        w = w.scaled(B=args.batch or w.B, H=args.heads or w.H)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
     else:

@@ -636,8 +636,10 @@ cudaError_t launch_attn_tc(const uint32_t* bq, const float* muq, const uint32_t*
     const int dv = dv_of(d);
     const int64_t ldv = round_up64(N, 16);
     const int vb = kernel_bias(bias_kind, gw);
-    // BA_QK_AUTO takes kind::i8 (the faster of the two on B200).
-    const bool f8 = variant == BA_QK_TC_F8;
+    // BA_QK_AUTO takes the faster kind per kernel, as measured on B200:
+    // kind::f8f6f4 (fp32 scores straight from TMEM, no integer conversion in
+    // the softmax) for the 128-key kernel, kind::i8 for the paired one.
+    const bool f8 = variant == BA_QK_TC_F8 || (variant == BA_QK_AUTO && !use_pair(bias_kind, B));
 
     CUtensorMap tv, tb;
     memset(&tv, 0, sizeof(tv));

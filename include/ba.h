@@ -62,7 +62,7 @@ typedef enum {
 
 /* How the binary Q.K contraction runs inside ba_attention_fwd_variant. */
 typedef enum {
-    BA_QK_AUTO = 0,        /* the library's fastest path for the shape (tcgen05 kind::i8) */
+    BA_QK_AUTO = 0,        /* the library's fastest path for the shape (tcgen05 kind::f8f6f4 or kind::i8) */
     BA_QK_POPC = 1,        /* CUDA cores: XOR + popcount on 32-bit words */
     BA_QK_MMA_B1 = 2,      /* warp mma.sync m16n8k128 .b1 XOR-popcount; PV by mma.sync u8 x s8 */
     BA_QK_TC_I8 = 3,       /* tcgen05 kind::i8, +-1 int8 operands, s32 in TMEM */
