@@ -21,8 +21,9 @@
 // Four launches, each one thread per query row or per key, the other side
 // streamed through shared memory in tiles of 32 tokens:
 //   bwd_stats_kernel : exact row maximum m, l = sum_j exp(S - m), D_i
-//   bwd_dq_kernel    : dq (and dbias, added with atomics)
-//   bwd_dk_kernel    : dk
+//   bwd_dq_kernel    : dq
+//   bwd_dk_kernel    : dk (and dbias, added with atomics: the lanes of a warp
+//                      hold consecutive keys, so the additions coalesce)
 //   bwd_dv_kernel    : dv
 // Scores are formed as in the forward's CUDA-core kernel:
 // S = (mu_q / sqrt(d)) mu_k z + b in fp32, z = d - 2 popcount(xor).
@@ -163,15 +164,17 @@ __device__ __forceinline__ void stage_keys(const Args& a, int64_t bh, int j0, ui
         }
 }
 
-// dq: one thread per query row.  dbias (optional) receives dS by atomics.
+// dq: one thread per query row.  A dense bias tile (the CTA's rows x TILE
+// keys) is staged through shared memory with coalesced loads.
 template <int W, typename InT>
 __global__ void __launch_bounds__(ROWS) bwd_dq_kernel(const Args a, const InT* __restrict__ q_raw, float clip,
-                                                      float* __restrict__ dq, float* __restrict__ dbias)
+                                                      float* __restrict__ dq)
 {
     constexpr int DC = 32 * W;
     __shared__ uint32_t s_k[TILE][W];
     __shared__ float s_mu[TILE];
     __shared__ __align__(16) float s_v[TILE][DC];
+    __shared__ float s_b[ROWS][TILE + 1];
     const int64_t bh = blockIdx.y;
     const int h = (int)(bh % a.H), N = a.N, d = a.d;
     const int i = blockIdx.x * ROWS + threadIdx.x;
@@ -190,15 +193,26 @@ __global__ void __launch_bounds__(ROWS) bwd_dq_kernel(const Args a, const InT* _
         ds[c] = 0.f;
     }
     float dmu = 0.f;
+    const int row0 = blockIdx.x * ROWS;
     for (int j0 = 0; j0 < N; j0 += TILE) {
         __syncthreads();
         stage_keys<W>(a, bh, j0, s_k, s_mu, s_v);
+        if (a.bias_kind == BA_BIAS_DENSE) {
+            // warp w loads rows w, w + 4, ...: each row's TILE keys are one 128-byte line
+            const int lane = threadIdx.x & 31;
+            for (int r = threadIdx.x >> 5; r < ROWS; r += ROWS / 32) {
+                const int ii = min(row0 + r, N - 1);
+                s_b[r][lane] = (j0 + lane < N) ? __ldg(a.bias + ((int64_t)h * N + ii) * a.bias_ld + j0 + lane) : 0.f;
+            }
+        }
         __syncthreads();
         const int nk = min(TILE, N - j0);
         for (int jj = 0; jj < nk; ++jj) {
             const int j = j0 + jj;
             const int z = zdot<W>(q, s_k[jj], d);
-            const float S = fmaf(cq * s_mu[jj], (float)z, bias_of(a.bias_kind, a.bias, a.bias_ld, h, N, a.gh, a.gw, ie, j));
+            const float bij = (a.bias_kind == BA_BIAS_DENSE) ? s_b[threadIdx.x][jj]
+                            : bias_of(a.bias_kind, a.bias, a.bias_ld, h, N, a.gh, a.gw, ie, j);
+            const float S = fmaf(cq * s_mu[jj], (float)z, bij);
             const float P = expf(S - m) * inv_l;
             float dp = 0.f;
 #pragma unroll
@@ -218,7 +232,6 @@ __global__ void __launch_bounds__(ROWS) bwd_dq_kernel(const Args a, const InT* _
 #pragma unroll
                 for (int b = 0; b < 32; ++b) ds[32 * w + b] += ((bits >> b) & 1u) ? dz : -dz;
             }
-            if (dbias != nullptr && ok) atomicAdd(dbias_at(a.bias_kind, dbias, a.bias_ld, h, N, a.gh, a.gw, i, j), dS);
         }
     }
     if (ok) {
@@ -259,10 +272,10 @@ __device__ __forceinline__ void stage_rows(const Args& a, int64_t bh, int i0, ui
     }
 }
 
-// dk: one thread per key.
+// dk: one thread per key; dbias (optional) receives dS by atomics.
 template <int W, typename InT>
 __global__ void __launch_bounds__(ROWS) bwd_dk_kernel(const Args a, const InT* __restrict__ k_raw, float clip,
-                                                      float* __restrict__ dk)
+                                                      float* __restrict__ dk, float* __restrict__ dbias)
 {
     constexpr int DC = 32 * W;
     __shared__ uint32_t s_q[TILE][W];
@@ -313,6 +326,7 @@ __global__ void __launch_bounds__(ROWS) bwd_dk_kernel(const Args a, const InT* _
 #pragma unroll
                 for (int b = 0; b < 32; ++b) dt[32 * w + b] += ((bits >> b) & 1u) ? dz : -dz;
             }
+            if (dbias != nullptr && ok) atomicAdd(dbias_at(a.bias_kind, dbias, a.bias_ld, h, N, a.gh, a.gw, i, j), dS);
         }
     }
     if (ok) {
@@ -387,9 +401,9 @@ cudaError_t launch_w(const Args& a, int BH, const InT* q, const InT* k, float cl
     bwd_stats_kernel<W><<<grid, ROWS, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, q, clip, dq, dbias);
+    bwd_dq_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, q, clip, dq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dk_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, k, clip, dk);
+    bwd_dk_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, k, clip, dk, dbias);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_dv_kernel<W><<<grid, ROWS, 0, st>>>(a, dv);
     return cudaGetLastError();
