@@ -20,6 +20,7 @@ operations / max-over-ranks time ("scaling": "weak": the per-GPU work is fixed).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -533,7 +534,8 @@ def run_ours(args, w, rank, local_rank, world):
         "device_status": status,
     }
     if not args.no_backward:
-        line["backward"] = time_backward(WORKLOADS["deit_b384"], dev)
+        bw = w if args.backward_workload == "main" else WORKLOADS[args.backward_workload]
+        line["backward"] = time_backward(bw, dev)
     if not args.no_side_workloads:
         # every rank times the same side workloads, so the ranks stay in step
         side = {}
@@ -730,10 +732,19 @@ def cpu_baseline(w, inp, budget_s=15.0, heads=1):
     t_attn = time.perf_counter() - t0
     BH = w.B * w.H
     t_full = t_pre * BH / heads + t_attn * (BH * N) / (heads * target)
+    # the DeiT-T workload (1 x 3 x 197 x 64) whole, on one core: the small
+    # correctness configuration, timed in full
+    wt = WORKLOADS["deit_t"]
+    it = make_inputs(wt)
+    t0 = time.perf_counter()
+    O.forward(it["q"], it["k"], it["v"], BIAS_KIND[wt.bias], it["bias"], it["ld"], nthreads=1)
+    t_small = time.perf_counter() - t0
     return {"value": w.ops / t_full / 1e12, "unit": "TOPS", "cores": used, "kind": "oracle",
             "sample": "%d head(s) x %d of %d query rows (all keys) + pre-passes of those heads, "
                       "%.1f s wall, scaled to the full workload" % (heads, target, N, t_pre + t_attn),
-            "seconds_full_workload_est": t_full}
+            "seconds_full_workload_est": t_full,
+            "deit_t_one_core": {"seconds": t_small, "tops": wt.ops / t_small / 1e12, "cores": 1,
+                                "sample": "the whole DeiT-T workload, pre-passes and forward"}}
 
 
 def run_reference(args, w, rank, world):
@@ -803,6 +814,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the training-side backward timing")
+    ap.add_argument("--backward-workload", default="deit_b384",
+                    help="workload of the backward timing ('main': the headline workload, after --batch/--heads)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiler captures)")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiler captures)")
@@ -814,6 +827,8 @@ def main(argv=None):
     rank, local_rank, world = dist_env()
     if args.workload in DECODE_WORKLOADS:
         w = DECODE_WORKLOADS[args.workload]
+        if args.batch or args.heads:
+            w = dataclasses.replace(w, B=args.batch or w.B, H=args.heads or w.H)
         if args.impl == "reference":
             line = run_reference_decode(args, w, rank, world)
         else:
