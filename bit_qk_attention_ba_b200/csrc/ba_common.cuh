@@ -16,6 +16,7 @@ enum : unsigned {
     kStatusTimeoutSoftmax  = 1u << 2,  // softmax warps gave up on a barrier
     kStatusTimeoutEpilogue = 1u << 3,
     kStatusBadLaunch       = 1u << 4,  // kernel found a launch shape it cannot serve
+    kStatusTimeoutCopy     = 1u << 5,  // a kernel gave up waiting for its bulk copies
 };
 
 __host__ __device__ inline int words_for(int d) { return (d + 31) / 32; }

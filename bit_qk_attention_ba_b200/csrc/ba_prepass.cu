@@ -21,6 +21,11 @@ cudaError_t launch_pack(const void* x, ba_dtype dt, int64_t tokens, int d, uint3
                         float* mu, cudaStream_t st, int sm_count);
 cudaError_t launch_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int8_t* vq,
                            float* sv, cudaStream_t st);
+bool prepass_tma_serves(int d, int esize);
+int prepass_tma_launches(int N);
+cudaError_t launch_prepass_tma(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H, int N, int d,
+                               uint32_t* bq, float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv,
+                               cudaStream_t st);
 
 namespace {
 
@@ -92,8 +97,9 @@ cudaError_t launch_fused_t(int nv, const void* q, const void* k, const void* v, 
 int prepass_launch_count(int N, int d, ba_dtype dt)
 {
     const int es = dt == BA_BF16 ? 2 : 4;
-    if (fused_vectors(N, d, es)) return 1;
     const bool v_one_block = (d * es) % 16 == 0 && vblock_smem_bytes(N, d) <= kVBlockMaxSmem;
+    if (prepass_tma_serves(d, es)) return prepass_tma_launches(N);
+    if (fused_vectors(N, d, es)) return 1;
     return 2 + (v_one_block ? 1 : 3);
 }
 
@@ -104,7 +110,13 @@ cudaError_t launch_prepass(const void* q, const void* k, const void* v, ba_dtype
     const int es = dt == BA_BF16 ? 2 : 4;
     const int nv = fused_vectors(N, d, es);
     const int BH = B * H;
-    if (nv && aligned(q, 16) && aligned(k, 16) && aligned(v, 16)) {
+    const bool al16 = aligned(q, 16) && aligned(k, 16) && aligned(v, 16);
+    if (al16 && prepass_tma_serves(d, es)) {
+        // 128-byte tokens: the TMA-fed kernel (ba_prepass_tma.cu).
+        const cudaError_t e = launch_prepass_tma(q, k, v, dt, B, H, N, d, bq, muq, bk, muk, vq, sv, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    if (nv && al16) {
         if (dt == BA_BF16)
             return launch_fused_t<__nv_bfloat16>(nv, q, k, v, BH, N, d, bq, muq, bk, muk, vq, sv, st);
         return launch_fused_t<float>(nv, q, k, v, BH, N, d, bq, muq, bk, muk, vq, sv, st);

@@ -14,9 +14,11 @@
 namespace ba {
 
 // One token held as NV 16-byte vectors (E = 16 / sizeof(T) channels each, so
-// d = NV E): the sign bits and the |x| sum are built in registers in channel
-// order, and mu = sum / d.  Every packing path ends here, so all of them give
-// the same bits and the same mu.
+// d = NV E): the sign bits are built in registers in channel order; the |x|
+// sum is pairwise in one fixed order (within a vector, then over the
+// vectors), which keeps the dependency chains short; mu = sum / d.  Every
+// packing path of the common head sizes ends here, so all of them give the
+// same bits and the same mu.
 template <typename T, int NV>
 __device__ __forceinline__ void pack_vectors(const uint4 (&raw)[NV], int d, uint32_t* __restrict__ bits,
                                              float* __restrict__ mu)
@@ -26,21 +28,31 @@ __device__ __forceinline__ void pack_vectors(const uint4 (&raw)[NV], int d, uint
     uint32_t w[W];
 #pragma unroll
     for (int i = 0; i < W; ++i) w[i] = 0u;
-    float s = 0.f;
+    float vs[NV];
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
         const T* v = reinterpret_cast<const T*>(&raw[k]);
+        float a[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) {
             const int c = k * E + e;
             const float f = to_f32<T>(v[e]);
             w[c >> 5] |= (f >= 0.f ? 1u : 0u) << (c & 31);
-            s += fabsf(f);
+            a[e] = fabsf(f);
         }
+#pragma unroll
+        for (int st = 1; st < E; st *= 2)
+#pragma unroll
+            for (int e = 0; e + st < E; e += 2 * st) a[e] += a[e + st];
+        vs[k] = a[0];
     }
 #pragma unroll
+    for (int st = 1; st < NV; st *= 2)
+#pragma unroll
+        for (int k = 0; k + st < NV; k += 2 * st) vs[k] += vs[k + st];
+#pragma unroll
     for (int i = 0; i < W; ++i) bits[i] = w[i];
-    *mu = __fdiv_rn(s, (float)d);
+    *mu = __fdiv_rn(vs[0], (float)d);
 }
 
 // One token read straight from global memory (its NV vectors in flight at once).

@@ -110,6 +110,39 @@ __global__ void vscale_kernel(float* sv, int64_t n)
     if (i < n) sv[i] = __fdiv_rn(sv[i], 127.0f);   // sv holds absmax bits == the float itself
 }
 
+// The tiled path's first half: zero sv, then fold every tile's channel
+// absmax into it as the bits of the (non-negative) floats.
+template <typename T>
+static cudaError_t launch_v_absmax_t(const void* v, int B, int H, int N, int d, float* sv, cudaStream_t st)
+{
+    const T* vp = static_cast<const T*>(v);
+    const int64_t BH = (int64_t)B * H;
+    cudaError_t e = cudaMemsetAsync(sv, 0, sizeof(float) * BH * d, st);
+    if (e != cudaSuccess) return e;
+    constexpr int E = 16 / sizeof(T);
+    const int rows = 512;
+    dim3 g1(ceil_div(N, rows), (unsigned)BH);
+    unsigned* amax = reinterpret_cast<unsigned*>(sv);
+    if (d % E == 0 && aligned(v, 16))
+        vabsmax_kernel<T, E><<<g1, 256, 0, st>>>(vp, N, d, rows, amax);
+    else
+        vabsmax_kernel<T, 1><<<g1, 256, 0, st>>>(vp, N, d, rows, amax);
+    return cudaGetLastError();
+}
+
+// The tiled path's last step: sv (absmax bits) -> scale = absmax / 127.
+cudaError_t launch_v_scale(float* sv, int64_t n, cudaStream_t st)
+{
+    vscale_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(sv, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_v_absmax(const void* v, ba_dtype dt, int B, int H, int N, int d, float* sv, cudaStream_t st)
+{
+    if (dt == BA_BF16) return launch_v_absmax_t<__nv_bfloat16>(v, B, H, N, d, sv, st);
+    return launch_v_absmax_t<float>(v, B, H, N, d, sv, st);
+}
+
 template <typename T>
 static cudaError_t launch_quant_v_t(const void* v, int B, int H, int N, int d, int8_t* vq, float* sv,
                                     cudaStream_t st)
@@ -126,21 +159,12 @@ static cudaError_t launch_quant_v_t(const void* v, int B, int H, int N, int d, i
         k<<<(unsigned)BH, 256, (size_t)small_smem, st>>>(vp, N, d, ldv, vq, sv);
         return cudaGetLastError();
     }
-    cudaError_t e = cudaMemsetAsync(sv, 0, sizeof(float) * BH * d, st);
+    cudaError_t e = launch_v_absmax_t<T>(v, B, H, N, d, sv, st);
     if (e != cudaSuccess) return e;
-    constexpr int E = 16 / sizeof(T);
-    const int rows = 512;
-    dim3 g1(ceil_div(N, rows), (unsigned)BH);
-    unsigned* amax = reinterpret_cast<unsigned*>(sv);
-    if (d % E == 0 && aligned(v, 16))
-        vabsmax_kernel<T, E><<<g1, 256, 0, st>>>(vp, N, d, rows, amax);
-    else
-        vabsmax_kernel<T, 1><<<g1, 256, 0, st>>>(vp, N, d, rows, amax);
     dim3 g2(ceil_div((int)ldv, 64), (unsigned)BH);
-    vquant_kernel<T><<<g2, 256, 0, st>>>(vp, N, d, ldv, amax, vq);
-    const int64_t n = BH * d;
-    vscale_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(sv, n);
-    return cudaGetLastError();
+    vquant_kernel<T><<<g2, 256, 0, st>>>(vp, N, d, ldv, reinterpret_cast<const unsigned*>(sv), vq);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? launch_v_scale(sv, BH * d, st) : e;
 }
 
 cudaError_t launch_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int8_t* vq,

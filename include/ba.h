@@ -105,14 +105,17 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
 /*
  * KD1 + KD3 in one call: the same outputs, bit for bit, as
  *   ba_pack_qk(q) -> bq, muq;  ba_pack_qk(k) -> bk, muk;  ba_quant_v(v) -> vq, sv
- * (layouts as above; q, k, v all [B, H, N, d] in dtype dt).  When the int8
- * codes of one (b, h) fit in 100 KB of shared memory (d (ba_vq_ld(N) + 4)
- * bytes), d size(dt) is a multiple of 16 bytes with d size(dt) / 16 in
- * {2, 4, 8, 9, 12, 16}, and q, k, v are 16-byte aligned, this is ONE kernel
- * launch: a CTA per (b, h) packs the head's query and key tokens, then
- * quantises its V (absmax sweep, then a code sweep transposed through shared
- * memory).  Otherwise the three passes run as separate launches.  Errors as
- * for the separate calls.
+ * (layouts as above; q, k, v all [B, H, N, d] in dtype dt), with q, k, v
+ * 16-byte aligned:
+ *   - 128-byte tokens (bf16 d = 64, fp32 d = 32): one launch fed by tensor
+ *     copies when ba_vq_ld(N) <= 1024; longer heads take three (V's channel
+ *     absmax, then Q, K and the V codes, then V's scales);
+ *   - otherwise ONE launch when the int8 codes of one (b, h) fit in 100 KB of
+ *     shared memory (d (ba_vq_ld(N) + 4) bytes) and d size(dt) / 16 is in
+ *     {2, 4, 8, 9, 12, 16}: a CTA per (b, h) packs the head's query and key
+ *     tokens, then quantises its V;
+ *   - otherwise the three passes as separate launches.
+ * Errors as for the separate calls.
  */
 ba_status ba_prepass_qkv(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H, int N, int d,
                          uint32_t* bq, float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv,

@@ -149,6 +149,12 @@ PREPASS_SHAPES = [
     (1, 2, 200, 128, "bf16"), (2, 2, 197, 64, "f32"), (1, 2, 50, 36, "f32"), (1, 2, 65, 48, "f32"),
     (1, 1, 90, 8, "f32"), (1, 2, 100, 72, "f32"), (1, 2, 90, 33, "f32"), (1, 1, 1500, 64, "bf16"),
     (1, 2, 2000, 64, "bf16"),
+    # 128-byte tokens (the TMA-fed kernel): one box, a unit of two boxes, a
+    # one-token unit after it, the largest head whose V it takes whole (1024
+    # code columns), one row past that (V absmax apart), and fp32 d = 32
+    (3, 2, 577, 64, "bf16"), (1, 3, 128, 64, "bf16"), (1, 3, 256, 64, "bf16"), (1, 2, 257, 64, "bf16"),
+    (2, 2, 1024, 64, "bf16"), (1, 2, 1025, 64, "bf16"), (2, 2, 197, 32, "f32"), (1, 1, 5, 32, "f32"),
+    (1, 2, 3000, 32, "f32"),
 ]
 
 
@@ -164,7 +170,10 @@ def test_prepass_shapes(shape):
     es = 2 if dtype == "bf16" else 4
     nv = d * es // 16 if (d * es) % 16 == 0 else 0
     fits = d * (ba.vq_ld(N) + 4) <= 100 * 1024      # the code tile of one (b, h) in shared memory
-    assert (ba.prepass_launches(N, d, tdt) == 1) == (nv in (2, 4, 8, 9, 12, 16) and fits)
+    if nv == 8:     # 128-byte tokens: one launch up to 1024 code columns, else three
+        assert ba.prepass_launches(N, d, tdt) == (1 if ba.vq_ld(N) <= 1024 else 3)
+    else:
+        assert (ba.prepass_launches(N, d, tdt) == 1) == (nv in (2, 4, 9, 12, 16) and fits)
 
 
 @pytest.mark.parametrize("N", [300, 5000])
