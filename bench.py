@@ -650,7 +650,7 @@ def run_decode(args, w, rank, local_rank, world):
             "traffic": recorded_traffic("decode_pv_kernel", os.path.join(CSRC, "ba_decode.cu"), w.name),
             "kernel_us": attn_t * 1e6,
             "peak_source": "measured HBM copy (%s)" % pk["src"], "algorithmic_bytes": nbytes,
-            "note": "events around ba_attention_decode: three launches (split maxima, codes + PV, combine)"}
+            "note": "events around ba_attention_decode: two launches (split maxima; codes, PV and the splits added by the last CTA of a head)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     line = {
         "metric": METRIC, "value": aggregate_tops(world, w.ops, ms), "unit": "TOPS", "n_gpus": world,
@@ -663,7 +663,7 @@ def run_decode(args, w, rank, local_rank, world):
                 "h2d_bytes_per_step": host_q.numel() * host_q.element_size(),
                 "d2h_bytes_per_step": host_out.numel() * host_out.element_size(), "ms_per_step": e2e_ms,
                 "cache": "resident on the device"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,            # pack the new queries, split maxima, codes + PV
         "clocks": clocks,
         "device_status": status,
     }

@@ -16,20 +16,25 @@
 // maxima, the next reduces them to the exact maximum m_i, quantises
 // P~ = exp(S - m_i) to u8 codes against it and forms each split's int32 PV
 // sums and P~ row sums; since every split quantises against the same m_i,
-// adding the splits' integer sums is exact.  A last launch adds the splits
-// and applies the epilogue O = sv acc / (255 l).
+// adding the splits' integer sums is exact.  The last split CTA of each head
+// to finish (an atomic ticket) adds the splits and applies the epilogue
+// O = sv acc / (255 l).  The second launch bulk-copies its split's V code
+// rows into shared memory first, so they stream in while the codes are formed.
 #include <math.h>
 
 #include <algorithm>
 
 #include "ba_common.cuh"
+#include "ba_sm100.cuh"
 
 namespace ba {
 namespace dec {
 
 constexpr int MAXQ = 16;          // query rows per head this path serves
 constexpr int THREADS = 256;
-constexpr int MAX_CHUNK = 2048;   // keys per split (u8 codes of 16 rows: 32 KB of shared memory)
+constexpr int MAX_CHUNK = 1024;   // keys per split
+constexpr int V_TILE = 64 * 1024; // at most this many V code bytes of a split in shared memory
+constexpr uint64_t kCopyWaitNs = 2000000000ull;
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct Params {
@@ -45,11 +50,23 @@ struct Params {
     int SA, CA;          // splits of the maximum sweep (wider: its per-key work is small)
     int bk_vec;          // key bits 4 W-byte aligned: one vector load per key (W = 2 or 4)
     int64_t ldv;
-    float* pmax;         // [BH][SA][MAXQ] row maxima of the maximum sweep's splits
-    float* psum;         // [BH][S][MAXQ] split sums of P~
-    int* pacc;           // [BH][S][MAXQ][d] int32 PV sums of each split
+    float* pmax;         // [BH][SA][Nq] row maxima of the maximum sweep's splits
+    float* psum;         // [BH][S][Nq] split sums of P~
+    int* pacc;           // [BH][S][Nq][d] int32 PV sums of each split
+    unsigned* ticket;    // [BH] split CTAs of the head done (zeroed by the maximum sweep)
     void* out;
+    int out_bf16;
+    unsigned* status;
 };
+
+// Row stride of a split's V codes in shared memory: C + 16 bytes, an odd
+// number of 16-byte chunks (C % 16 == 0), so 16-byte reads of consecutive
+// channels hit distinct bank groups.
+__host__ __device__ inline int v_stride(int C) { return C + 16; }
+
+// Dynamic shared memory of decode_pv_kernel: the split's V codes [d][C + 16],
+// the u8 P codes [Nq][C] and the int32 PV sums [Nq][d].
+__host__ __device__ inline int pv_smem_bytes(int d, int Nq, int C) { return d * v_stride(C) + Nq * C + Nq * d * 4; }
 
 __device__ __forceinline__ int dp4a_u8s8(uint32_t a_u8x4, uint32_t b_s8x4, int c)
 {
@@ -113,15 +130,15 @@ __device__ __forceinline__ float score(const Params& p, int h, const uint32_t (&
     return fmaf((float)(p.d - 2 * ham) * mk, cq[i], b);
 }
 
-// Block-wide reduction of MAXQ per-thread values (max or sum), lane order
+// Block-wide reduction of NQ per-thread values (max or sum), lane order
 // fixed; result in red[i] for every thread after the call.
-template <bool IS_MAX>
-__device__ __forceinline__ void block_reduce(float (&v)[MAXQ], int nq, float (&red)[THREADS / 32][MAXQ],
+template <bool IS_MAX, int NQ>
+__device__ __forceinline__ void block_reduce(float (&v)[NQ], int nq, float (&red)[THREADS / 32][MAXQ],
                                              float (&out)[MAXQ])
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int i = 0; i < MAXQ; ++i) {
+    for (int i = 0; i < NQ; ++i) {
         if (i >= nq) break;
         float x = v[i];
 #pragma unroll
@@ -141,8 +158,9 @@ __device__ __forceinline__ void block_reduce(float (&v)[MAXQ], int nq, float (&r
 }
 
 // Sweep 1: the row maxima of split blockIdx.x of head blockIdx.y.
-template <int W>
-__global__ void __launch_bounds__(THREADS)
+// NQ: the compile-time bound on the query rows (1, or MAXQ for 2 .. MAXQ).
+template <int W, int NQ>
+__global__ void __launch_bounds__(THREADS, 4)
 decode_max_kernel(const Params p)
 {
     __shared__ uint32_t qs[MAXQ][W];
@@ -152,168 +170,208 @@ decode_max_kernel(const Params p)
     const int s = blockIdx.x;
     const int64_t bh = blockIdx.y;
     const int h = (int)(bh % p.H);
+    if (s == 0 && threadIdx.x == 0) p.ticket[bh] = 0u;   // for the P.V launch after this one
     load_queries<W>(p, bh, qs, cq);
     __syncthreads();
-    float mx[MAXQ];
+    float mx[NQ];
 #pragma unroll
-    for (int i = 0; i < MAXQ; ++i) mx[i] = -INFINITY;
+    for (int i = 0; i < NQ; ++i) mx[i] = -INFINITY;
     const int j1 = min(p.Nk, (s + 1) * p.CA);
-#pragma unroll 8
-    for (int j = s * p.CA + threadIdx.x; j < j1; j += blockDim.x) {
-        uint32_t kb[W];
-        load_key<W>(p, bh, j, kb);
-        const float mk = __ldg(p.muk + bh * p.Nk + j);
+    // KB keys per thread in flight: their loads first, then the scores.
+    constexpr int KB = NQ == 1 ? 8 : 4;
+    for (int j = s * p.CA + threadIdx.x; j < j1; j += KB * blockDim.x) {
+        uint32_t kb[KB][W];
+        float mk[KB];
 #pragma unroll
-        for (int i = 0; i < MAXQ; ++i) {
-            if (i >= p.Nq) break;
-            mx[i] = fmaxf(mx[i], score<W>(p, h, kb, mk, qs, cq, i, j));
+        for (int u = 0; u < KB; ++u) {
+            const int ju = j + u * blockDim.x;
+            if (ju < j1) {
+                load_key<W>(p, bh, ju, kb[u]);
+                mk[u] = __ldg(p.muk + bh * p.Nk + ju);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < KB; ++u) {
+            const int ju = j + u * blockDim.x;
+            if (ju >= j1) break;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                if (i >= p.Nq) break;
+                mx[i] = fmaxf(mx[i], score<W>(p, h, kb[u], mk[u], qs, cq, i, ju));
+            }
         }
     }
-    block_reduce<true>(mx, p.Nq, red, res);
-    if (threadIdx.x < p.Nq) p.pmax[(bh * p.SA + s) * MAXQ + threadIdx.x] = res[threadIdx.x];
+    block_reduce<true, NQ>(mx, p.Nq, red, res);
+    if (threadIdx.x < p.Nq) p.pmax[(bh * p.SA + s) * p.Nq + threadIdx.x] = res[threadIdx.x];
 }
 
 // Sweep 2: exact m_i from the split maxima, u8 codes of this split's keys,
-// the split's P~ sums and int32 PV sums.
-template <int W>
+// the split's P~ sums and int32 PV sums.  The split's V code rows are
+// bulk-copied into shared memory first, so they stream in while the codes
+// are formed.
+template <int W, int NQ>
 __global__ void __launch_bounds__(THREADS, 3)
 decode_pv_kernel(const Params p)
 {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ __align__(8) uint64_t vbar;
     __shared__ uint32_t qs[MAXQ][W];
     __shared__ float cq[MAXQ];
     __shared__ float negm[MAXQ];
     __shared__ float red[THREADS / 32][MAXQ];
     __shared__ float res[MAXQ];
-    __shared__ __align__(16) uint8_t pq[MAXQ][MAX_CHUNK];
-    __shared__ int sacc[MAXQ][128];
     const int s = blockIdx.x;
     const int64_t bh = blockIdx.y;
     const int h = (int)(bh % p.H);
+    const int d = p.d;
+    const int j0 = s * p.C;
+    const int len = min(p.Nk - j0, p.C);
+    const int len16 = (len + 15) & ~15;       // <= ldv - j0: the copies stay inside the code rows
+    const int vst = v_stride(p.C);
+    uint8_t* vt = dsm;                        // [d][vst] V codes of keys j0 .. j0 + len16
+    uint8_t* pq = dsm + (size_t)d * vst;      // [Nq][C] u8 P codes
+    int* sacc = reinterpret_cast<int*>(pq + (size_t)p.Nq * p.C);   // [Nq][d] PV sums
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&vbar, 1);
+        sm100::fence_mbar_init();
+        sm100::mbar_arrive_expect_tx(&vbar, (uint32_t)(d * len16));
+    }
+    __syncthreads();
+    if (threadIdx.x < d)
+        sm100::bulk_load(vt + (size_t)threadIdx.x * vst, p.vq + (bh * d + threadIdx.x) * p.ldv + j0,
+                         (uint32_t)len16, &vbar);
     load_queries<W>(p, bh, qs, cq);
     if (threadIdx.x < p.Nq) {
         float m = -INFINITY;
-        for (int t = 0; t < p.SA; ++t) m = fmaxf(m, p.pmax[(bh * p.SA + t) * MAXQ + threadIdx.x]);
+        for (int t = 0; t < p.SA; ++t) m = fmaxf(m, p.pmax[(bh * p.SA + t) * p.Nq + threadIdx.x]);
         negm[threadIdx.x] = -m * LOG2E;
     }
-    for (int e = threadIdx.x; e < MAXQ * 128; e += blockDim.x) (&sacc[0][0])[e] = 0;
+    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) sacc[e] = 0;
     __syncthreads();
-    const int j0 = s * p.C;
-    const int len = min(p.Nk - j0, p.C);
-    const int len16 = (len + 15) & ~15;
-    float l[MAXQ];
+    float l[NQ];
 #pragma unroll
-    for (int i = 0; i < MAXQ; ++i) l[i] = 0.f;
-#pragma unroll 4
-    for (int jj = threadIdx.x; jj < len16; jj += blockDim.x) {
-        const int j = j0 + jj;
-        const bool live = jj < len;
-        uint32_t kb[W];
+    for (int i = 0; i < NQ; ++i) l[i] = 0.f;
+    // KB keys per thread in flight: their loads first, then the codes.
+    constexpr int KB = 4;
+    for (int jb = threadIdx.x; jb < len16; jb += KB * blockDim.x) {
+        uint32_t kb[KB][W];
+        float mk[KB];
 #pragma unroll
-        for (int w = 0; w < W; ++w) kb[w] = 0u;
-        if (live) load_key<W>(p, bh, j, kb);
-        const float mk = live ? __ldg(p.muk + bh * p.Nk + j) : 0.f;
+        for (int u = 0; u < KB; ++u) {
+            const int jj = jb + u * blockDim.x;
 #pragma unroll
-        for (int i = 0; i < MAXQ; ++i) {
-            if (i >= p.Nq) break;
-            uint32_t code = 0u;
-            if (live) {
-                const float pr = ex2(fmaf(score<W>(p, h, kb, mk, qs, cq, i, j), LOG2E, negm[i]));
-                l[i] += pr;
-                code = (uint32_t)__float2int_rn(255.f * pr);
+            for (int w = 0; w < W; ++w) kb[u][w] = 0u;
+            mk[u] = 0.f;
+            if (jj < len) {
+                load_key<W>(p, bh, j0 + jj, kb[u]);
+                mk[u] = __ldg(p.muk + bh * p.Nk + j0 + jj);
             }
-            pq[i][jj] = (uint8_t)code;
+        }
+#pragma unroll
+        for (int u = 0; u < KB; ++u) {
+            const int jj = jb + u * blockDim.x;
+            if (jj >= len16) break;
+            const bool live = jj < len;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                if (i >= p.Nq) break;
+                uint32_t code = 0u;
+                if (live) {
+                    const float pr = ex2(fmaf(score<W>(p, h, kb[u], mk[u], qs, cq, i, j0 + jj), LOG2E, negm[i]));
+                    l[i] += pr;
+                    code = (uint32_t)__float2int_rn(255.f * pr);
+                }
+                pq[i * p.C + jj] = (uint8_t)code;
+            }
         }
     }
-    block_reduce<false>(l, p.Nq, red, res);   // also orders the code writes before the reads below
-    if (threadIdx.x < p.Nq) p.psum[(bh * p.S + s) * MAXQ + threadIdx.x] = res[threadIdx.x];
+    block_reduce<false, NQ>(l, p.Nq, red, res);   // also orders the code writes before the reads below
+    if (threadIdx.x < p.Nq) p.psum[(bh * p.S + s) * p.Nq + threadIdx.x] = res[threadIdx.x];
+    // Every thread waits for the copies (none may land after the CTA ends).
+    const bool have_v = sm100::mbar_wait(&vbar, 0, nullptr, kCopyWaitNs);
+    if (!have_v && threadIdx.x == 0) atomicOr(p.status, kStatusTimeoutCopy);
 
     // PV: thread (g, c) takes channel c and key slice g of the split (G =
     // THREADS / d slices of whole 16-key groups), for every row; 16 keys per
-    // step: one 16-byte load of the channel's codes, one 16-byte read of each
+    // step: one 16-byte read of the channel's codes, one 16-byte read of each
     // row's P codes (the same address across the warp), four dp4a each.  The
     // slices' sums meet in shared memory (integer adds: order-free).
-    const int d = p.d;
     const int G = THREADS / d;
-    const bool pv_thread = threadIdx.x < G * d;
+    const bool pv_thread = have_v && threadIdx.x < G * d;
     const int c = threadIdx.x % d, g = threadIdx.x / d;
     const int groups = len16 / 16;
     const int k_lo = pv_thread ? 16 * (groups * g / G) : 0;
     const int k_hi = pv_thread ? 16 * (groups * (g + 1) / G) : 0;
-    int acc[MAXQ];
+    int acc[NQ];
 #pragma unroll
-    for (int i = 0; i < MAXQ; ++i) acc[i] = 0;
-    const int8_t* vrow = p.vq + (bh * d + c) * p.ldv + j0;
-    // Eight independent 16-byte loads of the channel's codes in flight per
-    // thread, then the rows' dot products.
-    constexpr int U = 8;
-    for (int k0 = k_lo; k0 < k_hi; k0 += 16 * U) {
-        uint4 vv[U];
+    for (int i = 0; i < NQ; ++i) acc[i] = 0;
+    const uint8_t* vrow = vt + (size_t)c * vst;
+#pragma unroll 2
+    for (int k = k_lo; k < k_hi; k += 16) {
+        const uint4 vv = *reinterpret_cast<const uint4*>(vrow + k);
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-            vv[u] = (k0 + 16 * u < k_hi) ? __ldg(reinterpret_cast<const uint4*>(vrow + k0 + 16 * u))
-                                         : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = k0 + 16 * u;
-            if (k >= k_hi) break;
-#pragma unroll
-            for (int i = 0; i < MAXQ; ++i) {
-                if (i >= p.Nq) break;
-                const uint4 a = *reinterpret_cast<const uint4*>(&pq[i][k]);
-                int t = acc[i];
-                t = dp4a_u8s8(a.x, vv[u].x, t);
-                t = dp4a_u8s8(a.y, vv[u].y, t);
-                t = dp4a_u8s8(a.z, vv[u].z, t);
-                acc[i] = dp4a_u8s8(a.w, vv[u].w, t);
-            }
+        for (int i = 0; i < NQ; ++i) {
+            if (i >= p.Nq) break;
+            const uint4 a = *reinterpret_cast<const uint4*>(pq + i * p.C + k);
+            int t = acc[i];
+            t = dp4a_u8s8(a.x, vv.x, t);
+            t = dp4a_u8s8(a.y, vv.y, t);
+            t = dp4a_u8s8(a.z, vv.z, t);
+            acc[i] = dp4a_u8s8(a.w, vv.w, t);
         }
     }
     if (pv_thread) {
 #pragma unroll
-        for (int i = 0; i < MAXQ; ++i) {
+        for (int i = 0; i < NQ; ++i) {
             if (i >= p.Nq) break;
-            atomicAdd(&sacc[i][c], acc[i]);
+            atomicAdd(&sacc[i * d + c], acc[i]);
         }
     }
     __syncthreads();
-    int* dst = p.pacc + ((bh * p.S + s) * MAXQ) * d;
-    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) dst[e] = sacc[e / d][e % d];
-}
+    int* dst = p.pacc + ((bh * p.S + s) * p.Nq) * d;
+    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) dst[e] = sacc[e];
 
-// The splits added (int64 code sums, P~ sums in split order) and the epilogue.
-template <typename OutT>
-__global__ void __launch_bounds__(THREADS)
-decode_combine_kernel(const Params p)
-{
-    const int64_t bh = blockIdx.x;
-    const int d = p.d;
-    OutT* out = static_cast<OutT*>(p.out);
+    // The head's last split CTA to finish adds the splits (int64 code sums,
+    // P~ sums in split order) and applies the epilogue O = sv acc / (255 l).
+    __shared__ unsigned s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&p.ticket[bh], 1u) == (unsigned)(p.S - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
     for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) {
-        const int i = e / d, c = e - i * d;
-        long long acc = 0;
-        float l = 0.f;
-        for (int s = 0; s < p.S; ++s) {
-            acc += p.pacc[((bh * p.S + s) * MAXQ + i) * d + c];
-            l += p.psum[(bh * p.S + s) * MAXQ + i];
+        const int i = e / d, c2 = e - i * d;
+        long long tot = 0;
+        float lt = 0.f;
+#pragma unroll 8
+        for (int t = 0; t < p.S; ++t) {
+            tot += __ldcg(p.pacc + ((bh * p.S + t) * p.Nq + i) * d + c2);
+            lt += __ldcg(p.psum + (bh * p.S + t) * p.Nq + i);
         }
-        const float o = __ldg(p.sv + bh * d + c) * (float)acc / (255.f * l);
-        if constexpr (sizeof(OutT) == 2) out[(bh * p.Nq + i) * d + c] = __float2bfloat16_rn(o);
-        else out[(bh * p.Nq + i) * d + c] = o;
+        const float o = __ldg(p.sv + bh * d + c2) * (float)tot / (255.f * lt);
+        const int64_t oi = (bh * p.Nq + i) * d + c2;
+        if (p.out_bf16) static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+        else static_cast<float*>(p.out)[oi] = o;
     }
 }
 
 // Splits per head: enough CTAs for about four per SM, at most MAX_CHUNK keys
-// and at least 256 keys per split (chunk lengths a multiple of 16).
+// (and at most V_TILE bytes of V codes) and at least 256 keys per split
+// (chunk lengths a multiple of 16).
 struct Split {
     int S, C;     // PV sweep: splits and keys per split
     int SA, CA;   // maximum sweep: four PV splits per split
 };
 
-inline Split choose_split(int64_t BH, int Nk, int sm_count)
+inline int max_chunk(int d) { return std::min(MAX_CHUNK, V_TILE / d / 16 * 16); }
+
+inline Split choose_split(int64_t BH, int Nk, int d, int sm_count)
 {
     const int64_t want = (4 * (int64_t)sm_count + BH - 1) / BH;
     int S = (int)std::max<int64_t>(1, std::min<int64_t>(want, (Nk + 255) / 256));
-    S = std::max(S, (Nk + MAX_CHUNK - 1) / MAX_CHUNK);
+    const int cmax = max_chunk(d);
+    S = std::max(S, (Nk + cmax - 1) / cmax);
     int C = (Nk + S - 1) / S;
     C = (C + 15) / 16 * 16;
     S = (Nk + C - 1) / C;
@@ -323,21 +381,27 @@ inline Split choose_split(int64_t BH, int Nk, int sm_count)
 
 inline int64_t workspace_bytes(int64_t BH, int Nk, int d, int sm_count)
 {
-    const Split sp = choose_split(BH, Nk, sm_count);
+    const Split sp = choose_split(BH, Nk, d, sm_count);
     const int64_t rows = BH * sp.S * MAXQ;
-    return rows * 4 * 2 + rows * d * 4;
+    return rows * 4 * 2 + rows * d * 4 + BH * 4;
+}
+
+template <int W, int NQ>
+cudaError_t launch_wq(Params p, int64_t BH, cudaStream_t st)
+{
+    decode_max_kernel<W, NQ><<<dim3(p.SA, (unsigned)BH), THREADS, 0, st>>>(p);
+    const int smem = pv_smem_bytes(p.d, p.Nq, p.C);
+    auto pv = decode_pv_kernel<W, NQ>;
+    cudaError_t e = cudaFuncSetAttribute(pv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    pv<<<dim3(p.S, (unsigned)BH), THREADS, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 template <int W>
-cudaError_t launch_w(Params p, int64_t BH, ba_dtype out_dt, cudaStream_t st)
+cudaError_t launch_w(Params p, int64_t BH, cudaStream_t st)
 {
-    decode_max_kernel<W><<<dim3(p.SA, (unsigned)BH), THREADS, 0, st>>>(p);
-    decode_pv_kernel<W><<<dim3(p.S, (unsigned)BH), THREADS, 0, st>>>(p);
-    if (out_dt == BA_BF16)
-        decode_combine_kernel<__nv_bfloat16><<<(unsigned)BH, THREADS, 0, st>>>(p);
-    else
-        decode_combine_kernel<float><<<(unsigned)BH, THREADS, 0, st>>>(p);
-    return cudaGetLastError();
+    return p.Nq == 1 ? launch_wq<W, 1>(p, BH, st) : launch_wq<W, MAXQ>(p, BH, st);
 }
 
 }  // namespace dec
@@ -353,7 +417,7 @@ cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, con
                                cudaStream_t st, int sm_count)
 {
     const int64_t BH = (int64_t)B * H;
-    const dec::Split sp = dec::choose_split(BH, Nk, sm_count);
+    const dec::Split sp = dec::choose_split(BH, Nk, d, sm_count);
     const int64_t rows = BH * sp.S * dec::MAXQ;
     dec::Params p;
     p.bq = bq; p.muq = muq; p.bk = bk; p.muk = muk; p.vq = vq; p.sv = sv;
@@ -365,12 +429,16 @@ cudaError_t launch_attn_decode(const uint32_t* bq, const float* muq, int Nq, con
     p.pmax = static_cast<float*>(workspace);
     p.psum = p.pmax + rows;
     p.pacc = reinterpret_cast<int*>(p.psum + rows);
+    p.ticket = reinterpret_cast<unsigned*>(p.pacc + rows * d);
     p.out = out;
+    p.out_bf16 = out_dt == BA_BF16;
+    p.status = device_status_ptr();
+    if (!p.status) return cudaErrorNotSupported;
     switch (words_for(d)) {
-        case 1: return dec::launch_w<1>(p, BH, out_dt, st);
-        case 2: return dec::launch_w<2>(p, BH, out_dt, st);
-        case 3: return dec::launch_w<3>(p, BH, out_dt, st);
-        default: return dec::launch_w<4>(p, BH, out_dt, st);
+        case 1: return dec::launch_w<1>(p, BH, st);
+        case 2: return dec::launch_w<2>(p, BH, st);
+        case 3: return dec::launch_w<3>(p, BH, st);
+        default: return dec::launch_w<4>(p, BH, st);
     }
 }
 

@@ -217,7 +217,7 @@ ba_status ba_attention_fwd_noalloc(const uint32_t* bq, const float* muq,
  * split over CTAs; every split quantises against the exact maximum, so the
  * splits' int32 sums add exactly.  workspace: device scratch of at least
  * ba_attention_decode_workspace_bytes(B, H, Nq, Nk, d) bytes, 256-byte
- * aligned, owned by the caller, rewritten by every call.  Three kernel
+ * aligned, owned by the caller, rewritten by every call.  Two kernel
  * launches on `stream`.
  */
 ba_status ba_attention_decode(const uint32_t* bq, const float* muq, int Nq,
