@@ -138,13 +138,23 @@ def _code_only(text):
     return re.sub(r"\s+", "", text)
 
 
+def _included(path, seen):
+    """path and every local header it includes ("..."), transitively, in order."""
+    path = os.path.normpath(path)
+    if path in seen or not os.path.exists(path):
+        return
+    seen.append(path)
+    for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', open(path).read(), flags=re.M):
+        _included(os.path.join(os.path.dirname(path), inc), seen)
+
+
 def source_hash(path):
-    """Hash of a kernel source and every shared kernel header (csrc/*.cuh),
+    """Hash of a kernel source and the local headers it includes (transitively),
     comments and whitespace removed: an edit of comments alone keeps a
-    recorded ncu summary valid, an edit of code in any header it may include
-    does not."""
-    parts = [path] + sorted(glob.glob(os.path.join(CSRC, "*.cuh")))
-    code = "".join(_code_only(open(p).read()) for p in parts if os.path.exists(p))
+    recorded ncu summary valid, an edit of code the kernel compiles does not."""
+    parts = []
+    _included(path, parts)
+    code = "".join(_code_only(open(p).read()) for p in parts)
     return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
