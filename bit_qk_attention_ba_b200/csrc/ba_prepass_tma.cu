@@ -1,5 +1,5 @@
-// ba_prepass_tma.cu -- the pre-pass for 128-byte tokens (bf16 d = 64, fp32
-// d = 32), fed by tensor-memory-accelerator copies.
+// ba_prepass_tma.cu -- the pre-pass for 128- and 144-byte tokens (bf16 d = 64
+// and 72, fp32 d = 32 and 36), fed by tensor-memory-accelerator copies.
 //
 // Method source: the paper-notes page "BinaryAttention: One-Bit QK-Attention
 // for Vision and Diffusion Transformers" (CVPR 2026), Key design 1 (sign bits
@@ -9,8 +9,9 @@
 // work is cut into small units and several CTAs share an SM.
 //
 // Rows reach shared memory as 128-row boxes of one 3-D tensor map per tensor
-// ([BH][N][128 bytes], 128-byte swizzle: the 16-byte chunk j of row r sits at
-// position j ^ (r & 7), which makes every access pattern below free of bank
+// ([BH][N][token bytes]; 128-byte rows with the 128-byte swizzle, the 16-byte
+// chunk j of row r at position j ^ (r & 7); 144-byte rows as they are, nine
+// chunks a row; either way every access pattern below is free of bank
 // conflicts; rows past the end of the head are zero-filled).  A CTA has
 // three box slots.  Work units, V first so the longest ones start in the first wave:
 //
@@ -24,7 +25,7 @@
 //   packed by pack_vectors (the routine of every packing path of these
 //   sizes), so the bits and mu equal those of the other paths, bit for bit.
 //
-// Codes: warp w takes the channels of chunk w, lane l the four keys
+// Codes: a warp takes the channels of one chunk, lane l the four keys
 // 4l .. 4l + 3 of a box, visited in a lane-dependent rotation (no bank
 // conflicts); each channel's four codes (vcode4, the rounding of every path)
 // are put back in key order by one byte permutation and go out as one word,
@@ -41,8 +42,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 256;
-constexpr int kBoxRows = 128;                 // rows per tensor copy (one box, 16 KB)
-constexpr int kBoxBytes = kBoxRows * 128;
+constexpr int kBoxRows = 128;                 // rows per tensor copy (one box)
 constexpr int kSlots = 3;                     // box slots of a CTA (copies in flight)
 constexpr int kUnitRows = kSlots * kBoxRows;  // rows of a Q, K or V-codes unit
 constexpr int kVWholeMaxLd = 1024;            // V of a head in one unit up to this code-row length
@@ -51,18 +51,27 @@ constexpr uint64_t kCopyWaitNs = 2000000000ull;
 enum : int { kVNone = 0, kVWhole = 1, kVCodes = 2 };
 
 struct PrepassMaps {
-    CUtensorMap q, k, v;                      // [BH][N][128 bytes], box (128 bytes, 128 rows, 1)
+    CUtensorMap q, k, v;                      // [BH][N][NV 16 bytes], box (NV 16 bytes, 128 rows, 1)
 };
 
+// Tokens of NV 16-byte chunks: 8 (128-byte rows, copied with the 128-byte
+// swizzle: chunk j of row r at position j ^ (r & 7)) or 9 (144-byte rows,
+// copied as they are: an odd number of chunks per row already spreads
+// consecutive rows over the bank groups).
+template <int NV> __host__ __device__ constexpr int box_bytes() { return kBoxRows * NV * 16; }
+template <int NV> __host__ __device__ constexpr int buf_align() { return NV == 8 ? 1024 : 128; }
+
+template <int NV>
 __device__ __forceinline__ uint4 ld_chunk(const uint8_t* box, int r, int j)
 {
-    return *reinterpret_cast<const uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4));
+    if constexpr (NV == 8) return *reinterpret_cast<const uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4));
+    else return *reinterpret_cast<const uint4*>(box + (r * NV + j) * 16);
 }
 
 // The codes of rows 4 lane .. 4 lane + 3 of one box for the E channels of
-// chunk w, written to vq rows (channel) at key offset key0 + 4 lane.
-template <typename T>
-__device__ __forceinline__ void codes_of_box(const uint8_t* box, int w, int lane, const float (&sc)[16 / sizeof(T)],
+// chunk cw, written to vq rows (channel) at key offset key0 + 4 lane.
+template <typename T, int NV>
+__device__ __forceinline__ void codes_of_box(const uint8_t* box, int cw, int lane, const float (&sc)[16 / sizeof(T)],
                                              const float (&rs)[16 / sizeof(T)], int8_t* vq_c0, int64_t ldv,
                                              int key0)
 {
@@ -73,7 +82,7 @@ __device__ __forceinline__ void codes_of_box(const uint8_t* box, int w, int lane
     const uint32_t sel = rot == 0 ? 0x3210u : rot == 1 ? 0x2103u : rot == 2 ? 0x1032u : 0x0321u;
     uint4 raw[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = ld_chunk(box, base + ((i + rot) & 3), w);
+    for (int i = 0; i < 4; ++i) raw[i] = ld_chunk<NV>(box, base + ((i + rot) & 3), cw);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const uint32_t word = vcode4(vec_elem<T>(raw[0], e), vec_elem<T>(raw[1], e), vec_elem<T>(raw[2], e),
@@ -82,16 +91,16 @@ __device__ __forceinline__ void codes_of_box(const uint8_t* box, int w, int lane
     }
 }
 
-// Channel absmax of the rows `rr + 32 j` (< nrows) of one box into m (bf16
-// pairs for bf16 input, as in vblock_quant, so the maxima are the same).
-template <typename T>
-__device__ __forceinline__ void absmax_of_box(const uint8_t* box, int cv, int rr, int nrows, uint32_t (&m)[4])
+// Channel absmax of chunk cv over the rows rr, rr + R, ... (< nrows) of one
+// box into m (bf16 pairs for bf16 input, as in vblock_quant, so the maxima
+// are the same).
+template <typename T, int NV>
+__device__ __forceinline__ void absmax_of_box(const uint8_t* box, int cv, int rr, int R, int nrows,
+                                              uint32_t (&m)[4])
 {
-#pragma unroll
-    for (int j = 0; j < kBoxRows / 32; ++j) {
-        const int r = rr + 32 * j;
-        if (r >= nrows) break;
-        const uint4 raw = ld_chunk(box, r, cv);
+    const int n = min(nrows, kBoxRows);
+    for (int r = rr; r < n; r += R) {
+        const uint4 raw = ld_chunk<NV>(box, r, cv);
         if constexpr (sizeof(T) == 2) {
             const uint32_t* h = &raw.x;
 #pragma unroll
@@ -109,20 +118,23 @@ __device__ __forceinline__ void absmax_of_box(const uint8_t* box, int cv, int rr
     }
 }
 
-template <typename T>
+template <typename T, int NV>
 __global__ void __launch_bounds__(kThreads, 4)
 prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64_t ldv, int nq, int vmode,
                    uint32_t* __restrict__ bq, float* __restrict__ muq, uint32_t* __restrict__ bk,
                    float* __restrict__ muk, int8_t* __restrict__ vq, float* __restrict__ sv,
                    unsigned* __restrict__ status)
 {
-    constexpr int E = 16 / sizeof(T);         // channels per 16-byte chunk; 8 chunks per token
+    constexpr int E = 16 / sizeof(T);         // channels per 16-byte chunk; NV chunks per token
+    constexpr int BB = box_bytes<NV>();
+    constexpr int RG = kThreads / NV;         // row groups of the absmax sweep (thread = (chunk, row group))
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kSlots];
-    __shared__ unsigned amax[64];
-    __shared__ float s_scale[64], s_rscale[64];
+    __shared__ unsigned amax[NV * E];
+    __shared__ float s_scale[NV * E], s_rscale[NV * E];
     __shared__ int s_fail;
-    uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + buf_align<NV>() - 1) &
+                                              ~uintptr_t(buf_align<NV>() - 1));
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int nbv = (int)((ldv + kBoxRows - 1) / kBoxRows);     // boxes of a head's V rows
     const int v_units = vmode == kVWhole ? 1 : vmode == kVCodes ? (int)((ldv + kUnitRows - 1) / kUnitRows) : 0;
@@ -152,14 +164,14 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
         fence_mbar_init();
         s_fail = 0;
     }
-    if (tid < 64) amax[tid] = 0u;
+    for (int c = tid; c < NV * E; c += kThreads) amax[c] = 0u;
     __syncthreads();
     // Copy i lands in slot i % kSlots (phase (i / kSlots) & 1): box i of the unit, or
     // for a streamed V box i % nbv of the head.
     auto issue = [&](int i) {
         const int b = streamed ? i % nbv : i;
-        mbar_arrive_expect_tx(&full[i % kSlots], (uint32_t)kBoxBytes);
-        tma_load_3d(buf + (i % kSlots) * kBoxBytes, map, &full[i % kSlots], 0, row0 + b * kBoxRows, (int)bh);
+        mbar_arrive_expect_tx(&full[i % kSlots], (uint32_t)BB);
+        tma_load_3d(buf + (i % kSlots) * BB, map, &full[i % kSlots], 0, row0 + b * kBoxRows, (int)bh);
     };
     if (tid == 0)
         for (int i = 0; i < min(boxes, kSlots); ++i) issue(i);
@@ -174,40 +186,42 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
         // ---------------------------------------------------- Q or K: a thread per token
         for (int t = tid; t < rows; t += kThreads) {
             if (!wait_copy(t / kBoxRows)) break;
-            const uint8_t* box = buf + (t / kBoxRows) * kBoxBytes;
+            const uint8_t* box = buf + (t / kBoxRows) * BB;
             const int r = t % kBoxRows;
-            uint4 raw[8];
+            uint4 raw[NV];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) raw[j] = ld_chunk(box, r, j);
+            for (int j = 0; j < NV; ++j) raw[j] = ld_chunk<NV>(box, r, j);
             const int64_t g = (int64_t)bh * N + row0 + t;
-            pack_vectors<T, 8>(raw, d, (kind == 0 ? bq : bk) + g * words_for(d), (kind == 0 ? muq : muk) + g);
+            pack_vectors<T, NV>(raw, d, (kind == 0 ? bq : bk) + g * words_for(d), (kind == 0 ? muq : muk) + g);
         }
         for (int i = 0; i < boxes; ++i) wait_copy(i);      // nothing may land after the CTA ends
     } else if (!streamed) {
         // ---------------------------------------------------- V codes, absmax given (bits of sv)
-        float sc[E], rs[E];
+        // Work items (box i, chunk cw) go round the warps.
+        for (int it = w; it < boxes * NV; it += kThreads / 32) {
+            const int i = it / NV, cw = it - i * NV;
+            float sc[E], rs[E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            sc[e] = __fdiv_rn(__uint_as_float(reinterpret_cast<const unsigned*>(sv)[bh * d + E * w + e]), 127.0f);
-            rs[e] = __frcp_rn(sc[e]);
+            for (int e = 0; e < E; ++e) {
+                sc[e] = __fdiv_rn(__uint_as_float(reinterpret_cast<const unsigned*>(sv)[bh * d + E * cw + e]), 127.0f);
+                rs[e] = __frcp_rn(sc[e]);
+            }
+            if (wait_copy(i))
+                codes_of_box<T, NV>(buf + i * BB, cw, lane, sc, rs, vq + ((size_t)bh * d + (size_t)E * cw) * ldv, ldv,
+                                    row0 + i * kBoxRows);
         }
-        int8_t* dst = vq + ((size_t)bh * d + (size_t)E * w) * ldv;
-        for (int i = 0; i < boxes; ++i)
-            if (wait_copy(i)) codes_of_box<T>(buf + i * kBoxBytes, w, lane, sc, rs, dst, ldv, row0 + i * kBoxRows);
+        for (int i = 0; i < boxes; ++i) wait_copy(i);
     } else {
         // ---------------------------------------------------- V of the whole head, two sweeps
         uint32_t m[4] = {0u, 0u, 0u, 0u};
-        const int cv = tid & 7, rr = tid >> 3;
-        float sc[E], rs[E];
-        int8_t* dst = vq + ((size_t)bh * d + (size_t)E * w) * ldv;
+        const int cv = tid % NV, rr = tid / NV;
         int issued = min(boxes, kSlots);
         for (int i = 0; i < boxes; ++i) {
             const bool have = i < issued && wait_copy(i);
-            const uint8_t* box = buf + (i % kSlots) * kBoxBytes;
+            const uint8_t* box = buf + (i % kSlots) * BB;
             if (i < nbv) {
-                if (have) absmax_of_box<T>(box, cv, rr, N - i * kBoxRows, m);
+                if (have && rr < RG) absmax_of_box<T, NV>(box, cv, rr, RG, N - i * kBoxRows, m);
                 if (i == nbv - 1) {
-                    // Fold the lanes l, l ^ 8, l ^ 16, l ^ 24 (same chunk), then the warps.
                     float mf[E];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -218,12 +232,18 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
                             mf[q] = __uint_as_float(m[q]);
                         }
                     }
+                    if constexpr (NV == 8) {
+                        // Fold the lanes l, l ^ 8, l ^ 16, l ^ 24 (same chunk), then the warps.
 #pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        unsigned u = __float_as_uint(mf[e]);
-                        u = max(u, __shfl_xor_sync(0xffffffffu, u, 8));
-                        u = max(u, __shfl_xor_sync(0xffffffffu, u, 16));
-                        if (lane < 8) atomicMax(&amax[E * cv + e], u);
+                        for (int e = 0; e < E; ++e) {
+                            unsigned u = __float_as_uint(mf[e]);
+                            u = max(u, __shfl_xor_sync(0xffffffffu, u, 8));
+                            u = max(u, __shfl_xor_sync(0xffffffffu, u, 16));
+                            if (lane < 8) atomicMax(&amax[E * cv + e], u);
+                        }
+                    } else if (rr < RG) {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) atomicMax(&amax[E * cv + e], __float_as_uint(mf[e]));
                     }
                     __syncthreads();
                     if (tid < d) {
@@ -233,14 +253,18 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
                         sv[bh * d + tid] = s;
                     }
                     __syncthreads();
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        sc[e] = s_scale[E * w + e];
-                        rs[e] = s_rscale[E * w + e];
-                    }
                 }
             } else if (have) {
-                codes_of_box<T>(box, w, lane, sc, rs, dst, ldv, (i - nbv) * kBoxRows);
+                for (int cw = w; cw < NV; cw += kThreads / 32) {
+                    float sc[E], rs[E];
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        sc[e] = s_scale[E * cw + e];
+                        rs[e] = s_rscale[E * cw + e];
+                    }
+                    codes_of_box<T, NV>(box, cw, lane, sc, rs, vq + ((size_t)bh * d + (size_t)E * cw) * ldv, ldv,
+                                        (i - nbv) * kBoxRows);
+                }
             }
             __syncthreads();                                // slot i % kSlots is free again
             if (!s_fail && i + kSlots < boxes) {
@@ -251,7 +275,7 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
     }
 }
 
-template <typename T>
+template <typename T, int NV>
 cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype dt, int BH, int N, int d, int vmode,
                          uint32_t* bq, float* muq, uint32_t* bk, float* muk, int8_t* vq, float* sv,
                          cudaStream_t st)
@@ -263,7 +287,7 @@ cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype d
     const int nq = ceil_div(N, kUnitRows);
     PrepassMaps maps;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {128u, (cuuint64_t)N * 128u};
+    const cuuint64_t strides[2] = {(cuuint64_t)NV * 16u, (cuuint64_t)N * NV * 16u};
     const cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)kBoxRows, 1u};
     const cuuint32_t es[3] = {1u, 1u, 1u};
     const CUtensorMapDataType ty = dt == BA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -271,11 +295,11 @@ cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype d
     CUtensorMap* dst[3] = {&maps.q, &maps.k, &maps.v};
     for (int i = 0; i < 3; ++i)
         if (encode(dst[i], ty, 3, const_cast<void*>(src[i]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   NV == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-    const int smem = kSlots * kBoxBytes + 1024;   // the box slots + slack to align them to 1024 bytes
-    auto kern = prepass_tma_kernel<T>;
+    const int smem = kSlots * box_bytes<NV>() + buf_align<NV>();   // the box slots + alignment slack
+    auto kern = prepass_tma_kernel<T, NV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int v_units = vmode == kVWhole ? 1 : vmode == kVCodes ? (int)((ldv + kUnitRows - 1) / kUnitRows) : 0;
@@ -290,10 +314,10 @@ cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype d
 cudaError_t launch_v_absmax(const void* v, ba_dtype dt, int B, int H, int N, int d, float* sv, cudaStream_t st);
 cudaError_t launch_v_scale(float* sv, int64_t n, cudaStream_t st);
 
-// Shapes the TMA pre-pass serves: 128-byte tokens.  V of a head in the same
-// launch up to 1024 code columns; longer heads take the channel absmax in a
-// launch before it and turn it into scales in one after it.
-bool prepass_tma_serves(int d, int esize) { return d * esize == 128; }
+// Shapes the TMA pre-pass serves: 128- and 144-byte tokens.  V of a head in
+// the same launch up to 1024 code columns; longer heads take the channel
+// absmax in a launch before it and turn it into scales in one after it.
+bool prepass_tma_serves(int d, int esize) { return d * esize == 128 || d * esize == 144; }
 int prepass_tma_launches(int N) { return round_up64(N, 16) <= kVWholeMaxLd ? 1 : 3; }
 
 // q, k, v 16-byte aligned.  cudaErrorNotSupported: nothing was launched.
@@ -312,8 +336,12 @@ cudaError_t launch_prepass_tma(const void* q, const void* k, const void* v, ba_d
         if (e != cudaSuccess) return e;
     }
     const int vmode = whole ? kVWhole : kVCodes;
-    e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
-                      : launch_tma_t<float>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);
+    if (d * es == 128)
+        e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16, 8>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
+                          : launch_tma_t<float, 8>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);
+    else
+        e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16, 9>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
+                          : launch_tma_t<float, 9>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);
     if (e == cudaSuccess && !whole) e = launch_v_scale(sv, (int64_t)BH * d, st);
     return e;
 }
