@@ -32,12 +32,27 @@ __device__ __forceinline__ void pack_vectors(const uint4 (&raw)[NV], int d, uint
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
         const T* v = reinterpret_cast<const T*>(&raw[k]);
+        if constexpr (sizeof(T) == 2) {
+            // The eight sign bits at once: an ordered x >= 0 on each bf16 pair
+            // (all ones per true half; -0 counts as >= 0, NaN does not), the
+            // halves' upper bytes gathered in channel order, each byte's low
+            // bit moved to bit i of a nibble by one multiply.
+            const uint32_t* h = &raw[k].x;
+            const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+            uint32_t m[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m[q] = __hge2_mask(*reinterpret_cast<const __nv_bfloat162*>(&h[q]), zero);
+            const uint32_t lo = __byte_perm(m[0], m[1], 0x7531), hi = __byte_perm(m[2], m[3], 0x7531);
+            const uint32_t b8 = (((lo & 0x01010101u) * 0x01020408u) >> 24) |
+                                ((((hi & 0x01010101u) * 0x01020408u) >> 24) << 4);
+            w[(k * E) >> 5] |= b8 << ((k * E) & 31);
+        }
         float a[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) {
             const int c = k * E + e;
             const float f = to_f32<T>(v[e]);
-            w[c >> 5] |= (f >= 0.f ? 1u : 0u) << (c & 31);
+            if constexpr (sizeof(T) != 2) w[c >> 5] |= (f >= 0.f ? 1u : 0u) << (c & 31);
             a[e] = fabsf(f);
         }
 #pragma unroll
