@@ -18,10 +18,11 @@
 //   dk_jc  = [|k_jc| <= clip] sum_i dz_ij s_ic + sign(k_jc) / d sum_i dS_ij mu_q,i z_ij / sqrt(d)
 //   dbias += dS (summed over the batch and over every (i, j) reading an entry)
 //
-// Four launches, each one thread per query row or per key, the other side
+// Four launches, each one thread per query row or per key (dq for d <= 32,
+// 64 or 128: two threads per row, each with half the channels), the other side
 // streamed through shared memory in tiles of 32 tokens:
 //   bwd_stats_kernel : exact row maximum m, l = sum_j exp(S - m), D_i
-//   bwd_dq_kernel    : dq
+//   bwd_dq2_kernel / bwd_dq_kernel : dq
 //   bwd_dk_kernel    : dk (and dbias, added with atomics: the lanes of a warp
 //                      hold consecutive keys, so the additions coalesce)
 //   bwd_dv_kernel    : dv
@@ -249,6 +250,110 @@ __global__ void __launch_bounds__(ROWS) bwd_dq_kernel(const Args a, const InT* _
     }
 }
 
+// dq with a row's channels split over two adjacent threads (half h takes
+// channels h DC / 2 .. (h + 1) DC / 2 - 1): half the accumulators per thread,
+// so twice the warps per SM; the two halves of dO . V^ meet by one shuffle.
+// For W = 1, 2, 4 (each half a whole number of sign words, or half a word).
+// The arithmetic of every (row, key, channel) is that of bwd_dq_kernel.
+template <int W, typename InT>
+__global__ void __launch_bounds__(ROWS) bwd_dq2_kernel(const Args a, const InT* __restrict__ q_raw, float clip,
+                                                       float* __restrict__ dq)
+{
+    constexpr int DC = 32 * W, HC = DC / 2, RPC = ROWS / 2;
+    constexpr int VS = DC + 4;                 // s_v row stride; the second half starts 4 floats later
+    static_assert(W == 1 || W == 2 || W == 4, "halves of whole sign words");
+    __shared__ uint32_t s_k[TILE][W];
+    __shared__ float s_mu[TILE];
+    __shared__ __align__(16) float s_v[TILE][VS];
+    __shared__ float s_b[RPC][TILE + 1];
+    const int64_t bh = blockIdx.y;
+    const int h = (int)(bh % a.H), N = a.N, d = a.d;
+    const int half = threadIdx.x & 1, lr = threadIdx.x >> 1;
+    const int c0 = half * HC;                  // first channel of this thread
+    const int vo = half * (HC + 4);            // where those channels sit in a row of s_v
+    const int i = blockIdx.x * RPC + lr;
+    const bool ok = i < N;
+    const int ie = ok ? i : N - 1;
+    uint32_t q[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) q[w] = __ldg(a.bq + (bh * N + ie) * W + w);
+    const float muq = __ldg(a.muq + bh * N + ie);
+    const float cq = muq * a.rsd;
+    const float m = a.m[bh * N + ie], inv_l = 1.f / a.l[bh * N + ie], Dv = a.D[bh * N + ie];
+    float g[HC], ds[HC];
+#pragma unroll
+    for (int cc = 0; cc < HC; ++cc) {
+        g[cc] = (c0 + cc < d) ? __ldg(a.dout + (bh * N + ie) * d + c0 + cc) : 0.f;
+        ds[cc] = 0.f;
+    }
+    float dmu = 0.f;
+    const int row0 = blockIdx.x * RPC;
+    for (int j0 = 0; j0 < N; j0 += TILE) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < TILE * W; e += ROWS) {
+            const int r = e / W, w = e - r * W;
+            s_k[r][w] = (j0 + r < N) ? __ldg(a.bk + (bh * N + j0 + r) * W + w) : 0u;
+        }
+        for (int r = threadIdx.x; r < TILE; r += ROWS) s_mu[r] = (j0 + r < N) ? __ldg(a.muk + bh * N + j0 + r) : 0.f;
+        for (int e = threadIdx.x; e < TILE * DC; e += ROWS) {
+            const int c = e / TILE, r = e - c * TILE;      // consecutive threads: consecutive keys of a channel
+            float val = 0.f;
+            if (c < d && j0 + r < N) val = __ldg(a.sv + bh * d + c) * (float)a.vq[(bh * d + c) * a.ldv + j0 + r];
+            s_v[r][c + (c >= HC ? 4 : 0)] = val;
+        }
+        if (a.bias_kind == BA_BIAS_DENSE) {
+            const int lane = threadIdx.x & 31;
+            for (int r = threadIdx.x >> 5; r < RPC; r += ROWS / 32) {
+                const int ii = min(row0 + r, N - 1);
+                s_b[r][lane] = (j0 + lane < N) ? __ldg(a.bias + ((int64_t)h * N + ii) * a.bias_ld + j0 + lane) : 0.f;
+            }
+        }
+        __syncthreads();
+        const int nk = min(TILE, N - j0);
+        for (int jj = 0; jj < nk; ++jj) {
+            const int j = j0 + jj;
+            const int z = zdot<W>(q, s_k[jj], d);
+            const float bij = (a.bias_kind == BA_BIAS_DENSE) ? s_b[lr][jj]
+                            : bias_of(a.bias_kind, a.bias, a.bias_ld, h, N, a.gh, a.gw, ie, j);
+            const float S = fmaf(cq * s_mu[jj], (float)z, bij);
+            const float P = expf(S - m) * inv_l;
+            float dp = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < HC; cc += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(&s_v[jj][vo + cc]);
+                dp = fmaf(g[cc], v4.x, dp);
+                dp = fmaf(g[cc + 1], v4.y, dp);
+                dp = fmaf(g[cc + 2], v4.z, dp);
+                dp = fmaf(g[cc + 3], v4.w, dp);
+            }
+            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+            const float dS = P * (dp - Dv);
+            dmu = fmaf(dS * s_mu[jj], (float)z, dmu);
+            const float dz = dS * cq * s_mu[jj];
+#pragma unroll
+            for (int w = 0; w < (W == 1 ? 1 : W / 2); ++w) {
+                const uint32_t bits = (W == 1) ? (s_k[jj][0] >> (16 * half)) : s_k[jj][half * (W / 2) + w];
+#pragma unroll
+                for (int b = 0; b < (W == 1 ? 16 : 32); ++b) ds[32 * w + b] += ((bits >> b) & 1u) ? dz : -dz;
+            }
+        }
+    }
+    if (ok) {
+        const float dmuq = dmu * a.rsd / (float)d;     // d mu / d q_c = sign(q_c) / d
+        const InT* xr = q_raw + (bh * N + i) * d;
+        float* dst = dq + (bh * N + i) * d;
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc) {
+            const int c = c0 + cc;
+            if (c < d) {
+                const float x = ld_val<InT>(xr + c);
+                const float sgn = ((q[c >> 5] >> (c & 31)) & 1u) ? 1.f : -1.f;
+                dst[c] = (fabsf(x) <= clip ? ds[cc] : 0.f) + dmuq * sgn;
+            }
+        }
+    }
+}
+
 // Stage TILE query rows of head bh: bits, scales, row statistics, dO rows.
 template <int W>
 __device__ __forceinline__ void stage_rows(const Args& a, int64_t bh, int i0, uint32_t (*s_q)[W], float* s_mu,
@@ -401,7 +506,12 @@ cudaError_t launch_w(const Args& a, int BH, const InT* q, const InT* k, float cl
     bwd_stats_kernel<W><<<grid, ROWS, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, q, clip, dq);
+    if constexpr (W == 3) {
+        bwd_dq_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, q, clip, dq);
+    } else {
+        dim3 grid2(ceil_div(a.N, ROWS / 2), BH);
+        bwd_dq2_kernel<W, InT><<<grid2, ROWS, 0, st>>>(a, q, clip, dq);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_dk_kernel<W, InT><<<grid, ROWS, 0, st>>>(a, k, clip, dk, dbias);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
