@@ -376,3 +376,38 @@ def test_attention_full_size(name, variant):
 
 def test_device_status_is_clean():
     assert ba.check_device_status() == 0
+
+
+MISALIGNED_SHAPES = [(2, 2, 577, 64, "bf16"), (1, 2, 300, 72, "bf16"), (2, 2, 197, 32, "f32"), (1, 1, 1025, 64, "bf16")]
+
+
+@pytest.mark.parametrize("shape", MISALIGNED_SHAPES, ids=["x".join(map(str, s)) for s in MISALIGNED_SHAPES])
+def test_prepass_misaligned_inputs(shape):
+    """q, k, v one element past a 16-byte boundary (element-aligned, as the
+    ABI allows) cannot take the tensor-copy or fused paths; the passes they
+    fall back to give the same bits, codes and scales, and mu within fp32
+    summation error (the fallback adds |x| in another fixed order)."""
+    B, H, N, d, dtype = shape
+    w = Workload("pp", B, H, N, d, dtype=dtype)
+    inp = make_inputs(w)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+
+    def misaligned(x):
+        flat = torch.from_numpy(x).to(tdt).reshape(-1)
+        buf = torch.zeros(flat.numel() + 1, dtype=tdt, device=DEV)
+        view = buf[1:].view(x.shape)
+        view.copy_(flat.view(x.shape).to(DEV))
+        assert view.data_ptr() % 16 != 0
+        return view
+
+    aligned = [_gpu(inp[n], dtype) for n in ("q", "k", "v")]
+    shifted = [misaligned(inp[n]) for n in ("q", "k", "v")]
+    want = ba.prepass_qkv(*aligned)
+    got = ba.prepass_qkv(*shifted)
+    torch.cuda.synchronize()
+    for idx in (0, 2, 4, 5):                       # bq, bk, vq, sv
+        assert torch.equal(want[idx], got[idx])
+    for idx in (1, 3):                             # muq, muk
+        a, b = want[idx].double(), got[idx].double()
+        assert ((a - b).abs() / a.abs().clamp_min(1e-30)).max().item() <= d * 2.0 ** -24 + 2.0 ** -23
+    assert ba.check_device_status() == 0
