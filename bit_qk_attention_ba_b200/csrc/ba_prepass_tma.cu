@@ -1,5 +1,6 @@
-// ba_prepass_tma.cu -- the pre-pass for 128- and 144-byte tokens (bf16 d = 64
-// and 72, fp32 d = 32 and 36), fed by tensor-memory-accelerator copies.
+// ba_prepass_tma.cu -- the pre-pass for 128-, 144- and 256-byte tokens (bf16
+// d = 64, 72 and 128, fp32 d = 32, 36 and 64), fed by tensor-memory-accelerator
+// copies.
 //
 // Method source: the paper-notes page "BinaryAttention: One-Bit QK-Attention
 // for Vision and Diffusion Transformers" (CVPR 2026), Key design 1 (sign bits
@@ -55,17 +56,35 @@ struct PrepassMaps {
 };
 
 // Tokens of NV 16-byte chunks: 8 (128-byte rows, copied with the 128-byte
-// swizzle: chunk j of row r at position j ^ (r & 7)) or 9 (144-byte rows,
+// swizzle: chunk j of row r at position j ^ (r & 7)), 9 (144-byte rows,
 // copied as they are: an odd number of chunks per row already spreads
-// consecutive rows over the bank groups).
+// consecutive rows over the bank groups) or 16 (each token two 128-byte rows
+// 2r and 2r + 1 of a 4-D copy, swizzled as the 128-byte rows are).
 template <int NV> __host__ __device__ constexpr int box_bytes() { return kBoxRows * NV * 16; }
-template <int NV> __host__ __device__ constexpr int buf_align() { return NV == 8 ? 1024 : 128; }
+template <int NV> __host__ __device__ constexpr int buf_align() { return NV == 9 ? 128 : 1024; }
 
 template <int NV>
 __device__ __forceinline__ uint4 ld_chunk(const uint8_t* box, int r, int j)
 {
-    if constexpr (NV == 8) return *reinterpret_cast<const uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4));
-    else return *reinterpret_cast<const uint4*>(box + (r * NV + j) * 16);
+    if constexpr (NV == 8) {
+        return *reinterpret_cast<const uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4));
+    } else if constexpr (NV == 16) {
+        const int row = 2 * r + (j >> 3);
+        return *reinterpret_cast<const uint4*>(box + row * 128 + (((j & 7) ^ (row & 7)) << 4));
+    } else {
+        return *reinterpret_cast<const uint4*>(box + (r * NV + j) * 16);
+    }
+}
+
+// A 4-D tensor copy (the 256-byte tokens' map: 128-byte half, half, row, head).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)),
+          "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
 }
 
 // The codes of rows 4 lane .. 4 lane + 3 of one box for the E channels of
@@ -171,7 +190,10 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
     auto issue = [&](int i) {
         const int b = streamed ? i % nbv : i;
         mbar_arrive_expect_tx(&full[i % kSlots], (uint32_t)BB);
-        tma_load_3d(buf + (i % kSlots) * BB, map, &full[i % kSlots], 0, row0 + b * kBoxRows, (int)bh);
+        if constexpr (NV == 16)
+            tma_load_4d(buf + (i % kSlots) * BB, map, &full[i % kSlots], 0, 0, row0 + b * kBoxRows, (int)bh);
+        else
+            tma_load_3d(buf + (i % kSlots) * BB, map, &full[i % kSlots], 0, row0 + b * kBoxRows, (int)bh);
     };
     if (tid == 0)
         for (int i = 0; i < min(boxes, kSlots); ++i) issue(i);
@@ -232,14 +254,14 @@ prepass_tma_kernel(const __grid_constant__ PrepassMaps maps, int N, int d, int64
                             mf[q] = __uint_as_float(m[q]);
                         }
                     }
-                    if constexpr (NV == 8) {
-                        // Fold the lanes l, l ^ 8, l ^ 16, l ^ 24 (same chunk), then the warps.
+                    if constexpr (NV == 8 || NV == 16) {
+                        // Fold the lanes that share the chunk (l, l ^ NV, ...), then the warps.
 #pragma unroll
                         for (int e = 0; e < E; ++e) {
                             unsigned u = __float_as_uint(mf[e]);
-                            u = max(u, __shfl_xor_sync(0xffffffffu, u, 8));
-                            u = max(u, __shfl_xor_sync(0xffffffffu, u, 16));
-                            if (lane < 8) atomicMax(&amax[E * cv + e], u);
+#pragma unroll
+                            for (int o = NV; o < 32; o *= 2) u = max(u, __shfl_xor_sync(0xffffffffu, u, o));
+                            if (lane < NV) atomicMax(&amax[E * cv + e], u);
                         }
                     } else if (rr < RG) {
 #pragma unroll
@@ -286,16 +308,26 @@ cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype d
     const int64_t ldv = round_up64(N, 16);
     const int nq = ceil_div(N, kUnitRows);
     PrepassMaps maps;
-    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)NV * 16u, (cuuint64_t)N * NV * 16u};
-    const cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)kBoxRows, 1u};
-    const cuuint32_t es[3] = {1u, 1u, 1u};
+    // [BH][N][token]; 256-byte tokens as [BH][N][2][128 bytes] (4-D), so each
+    // half is a 128-byte row the swizzle applies to.
+    const int rank = NV == 16 ? 4 : 3;
+    const cuuint64_t inner = NV == 16 ? (cuuint64_t)d / 2 : (cuuint64_t)d;
+    const cuuint64_t dims3[3] = {inner, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t dims4[4] = {inner, 2u, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t strides3[2] = {(cuuint64_t)NV * 16u, (cuuint64_t)N * NV * 16u};
+    const cuuint64_t strides4[3] = {128u, (cuuint64_t)NV * 16u, (cuuint64_t)N * NV * 16u};
+    const cuuint32_t box3[3] = {(cuuint32_t)inner, (cuuint32_t)kBoxRows, 1u};
+    const cuuint32_t box4[4] = {(cuuint32_t)inner, 2u, (cuuint32_t)kBoxRows, 1u};
+    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    const cuuint64_t* dims = NV == 16 ? dims4 : dims3;
+    const cuuint64_t* strides = NV == 16 ? strides4 : strides3;
+    const cuuint32_t* box = NV == 16 ? box4 : box3;
     const CUtensorMapDataType ty = dt == BA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const void* src[3] = {q, k, v};
     CUtensorMap* dst[3] = {&maps.q, &maps.k, &maps.v};
     for (int i = 0; i < 3; ++i)
-        if (encode(dst[i], ty, 3, const_cast<void*>(src[i]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   NV == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        if (encode(dst[i], ty, rank, const_cast<void*>(src[i]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   NV == 9 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     const int smem = kSlots * box_bytes<NV>() + buf_align<NV>();   // the box slots + alignment slack
@@ -314,10 +346,10 @@ cudaError_t launch_tma_t(const void* q, const void* k, const void* v, ba_dtype d
 cudaError_t launch_v_absmax(const void* v, ba_dtype dt, int B, int H, int N, int d, float* sv, cudaStream_t st);
 cudaError_t launch_v_scale(float* sv, int64_t n, cudaStream_t st);
 
-// Shapes the TMA pre-pass serves: 128- and 144-byte tokens.  V of a head in
+// Shapes the TMA pre-pass serves: 128-, 144- and 256-byte tokens.  V of a head in
 // the same launch up to 1024 code columns; longer heads take the channel
 // absmax in a launch before it and turn it into scales in one after it.
-bool prepass_tma_serves(int d, int esize) { return d * esize == 128 || d * esize == 144; }
+bool prepass_tma_serves(int d, int esize) { return d * esize == 128 || d * esize == 144 || d * esize == 256; }
 int prepass_tma_launches(int N) { return round_up64(N, 16) <= kVWholeMaxLd ? 1 : 3; }
 
 // q, k, v 16-byte aligned.  cudaErrorNotSupported: nothing was launched.
@@ -339,6 +371,9 @@ cudaError_t launch_prepass_tma(const void* q, const void* k, const void* v, ba_d
     if (d * es == 128)
         e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16, 8>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
                           : launch_tma_t<float, 8>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);
+    else if (d * es == 256)
+        e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16, 16>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
+                          : launch_tma_t<float, 16>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);
     else
         e = dt == BA_BF16 ? launch_tma_t<__nv_bfloat16, 9>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st)
                           : launch_tma_t<float, 9>(q, k, v, dt, BH, N, d, vmode, bq, muq, bk, muk, vq, sv, st);

@@ -107,9 +107,10 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d,
  *   ba_pack_qk(q) -> bq, muq;  ba_pack_qk(k) -> bk, muk;  ba_quant_v(v) -> vq, sv
  * (layouts as above; q, k, v all [B, H, N, d] in dtype dt), with q, k, v
  * 16-byte aligned:
- *   - 128- and 144-byte tokens (bf16 d = 64 or 72, fp32 d = 32 or 36): one
- *     launch fed by tensor copies when ba_vq_ld(N) <= 1024; longer heads take
- *     three (V's channel absmax, then Q, K and the V codes, then V's scales);
+ *   - 128-, 144- and 256-byte tokens (bf16 d = 64, 72 or 128, fp32 d = 32, 36
+ *     or 64): one launch fed by tensor copies when ba_vq_ld(N) <= 1024; longer
+ *     heads take three (V's channel absmax, then Q, K and the V codes, then V's
+ *     scales);
  *   - otherwise ONE launch when the int8 codes of one (b, h) fit in 100 KB of
  *     shared memory (d (ba_vq_ld(N) + 4) bytes) and d size(dt) / 16 is in
  *     {2, 4, 8, 9, 12, 16}: a CTA per (b, h) packs the head's query and key

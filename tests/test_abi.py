@@ -51,8 +51,8 @@ def test_pure_helpers(lib):
 def test_prepass_launch_count(lib):
     """One fused launch when a (b, h) block of V fits in shared memory and the
     token is 2, 4, 8, 9, 12 or 16 vectors of 16 bytes; else pack Q, pack K and
-    one (one-block V) or three (tiled V) quantiser launches.  128-byte tokens
-    and 144-byte tokens take one launch up to 1024 code columns, else three
+    one (one-block V) or three (tiled V) quantiser launches.  128-, 144- and
+    256-byte tokens take one launch up to 1024 code columns, else three
     (V's absmax, then Q, K and the V codes, then V's scales)."""
     bf16, f32 = 1, 0
     assert lib.ba_prepass_launches(577, 64, bf16) == 1        # DeiT-B/384
@@ -64,7 +64,8 @@ def test_prepass_launch_count(lib):
     assert lib.ba_prepass_launches(1025, 64, bf16) == 3
     assert lib.ba_prepass_launches(1500, 32, f32) == 3
     assert lib.ba_prepass_launches(16384, 72, bf16) == 3      # 144-byte tokens
-    assert lib.ba_prepass_launches(16384, 64, f32) == 5       # 256-byte tokens
+    assert lib.ba_prepass_launches(16384, 64, f32) == 3       # 256-byte tokens
+    assert lib.ba_prepass_launches(16384, 48, f32) == 5       # 192-byte tokens: separate passes, V tiled
     assert lib.ba_prepass_launches(90, 33, f32) == 5          # d * 4 not a multiple of 16
     assert lib.ba_prepass_launches(0, 64, bf16) == -1
     assert lib.ba_prepass_launches(8, 129, bf16) == -1

@@ -158,6 +158,9 @@ PREPASS_SHAPES = [
     # 144-byte tokens (nine 16-byte chunks, no swizzle): whole-head V and V
     # absmax apart, bf16 d = 72 and fp32 d = 36
     (2, 2, 577, 72, "bf16"), (1, 3, 1025, 72, "bf16"), (2, 2, 197, 36, "f32"), (1, 1, 3000, 36, "f32"),
+    # 256-byte tokens (two swizzled 128-byte rows each): bf16 d = 128 with V's
+    # absmax apart, fp32 d = 64 over three units
+    (1, 2, 1025, 128, "bf16"), (1, 1, 2000, 64, "f32"),
 ]
 
 
@@ -173,10 +176,10 @@ def test_prepass_shapes(shape):
     es = 2 if dtype == "bf16" else 4
     nv = d * es // 16 if (d * es) % 16 == 0 else 0
     fits = d * (ba.vq_ld(N) + 4) <= 100 * 1024      # the code tile of one (b, h) in shared memory
-    if nv in (8, 9):    # 128- and 144-byte tokens: one launch up to 1024 code columns, else three
+    if nv in (8, 9, 16):    # 128-, 144- and 256-byte tokens: one launch up to 1024 code columns, else three
         assert ba.prepass_launches(N, d, tdt) == (1 if ba.vq_ld(N) <= 1024 else 3)
     else:
-        assert (ba.prepass_launches(N, d, tdt) == 1) == (nv in (2, 4, 12, 16) and fits)
+        assert (ba.prepass_launches(N, d, tdt) == 1) == (nv in (2, 4, 12) and fits)
 
 
 @pytest.mark.parametrize("N", [300, 5000])
