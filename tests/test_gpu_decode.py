@@ -73,6 +73,11 @@ SHAPES = [
     (1, 2, 7, 2049, 32, "f32", True),
     (1, 1, 2, 70001, 64, "bf16", False),
     (3, 1, 16, 33, 1, "f32", True),
+    # one query row (the kernels' one-row instances) for every sign-word count
+    (1, 2, 1, 4097, 128, "f32", True),
+    (2, 2, 1, 777, 72, "bf16", False),
+    (1, 3, 1, 20000, 32, "bf16", True),
+    (2, 1, 1, 33, 1, "f32", False),
 ]
 
 
