@@ -161,6 +161,8 @@ PREPASS_SHAPES = [
     # 256-byte tokens (two swizzled 128-byte rows each): bf16 d = 128 with V's
     # absmax apart, fp32 d = 64 over three units
     (1, 2, 1025, 128, "bf16"), (1, 1, 2000, 64, "f32"),
+    # a one-token head for each token width (a 128-row box over one row)
+    (1, 2, 1, 72, "bf16"), (1, 2, 1, 64, "f32"), (2, 1, 1, 128, "bf16"),
 ]
 
 
