@@ -51,6 +51,7 @@
 // in the device status word, tells the other roles to stop, lets issued copies
 // and tensor-core work drain, frees TMEM and returns.
 #include "ba_attn_tc_common.cuh"
+#include "ba_tc_warp.cuh"
 
 namespace ba {
 
@@ -200,11 +201,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
 
     if (warp == LOAD_WARP) {
         // ---------------------------------------------------------------- loader
-        // One thread fills stage u % S for step u: the staged key tile, the
-        // bias of the step (the window of a reversed table row in four shifted
-        // copies, or four dense-bias boxes), and in pass B two V boxes.  All
-        // copies complete on the stage's FULL barrier.
-        if (lane == 0) {
+        // The warp fills stage u % S for step u (uniform loop, one elected
+        // lane issuing the copies in order, key tile first): the staged key
+        // tile, the bias of the step (the window of a reversed table row in
+        // four shifted copies, or four dense-bias boxes), and in pass B two V
+        // boxes.  All copies complete on the stage's FULL barrier.
+        {
             const size_t row_len = 2 * (size_t)p.gw;
             const float* rps_h = (BIAS == BIAS_RP_FAST) ? p.rps + (size_t)h * (2 * p.gh - 1) * 4 * row_len : nullptr;
             const int ri = (BIAS == BIAS_RP_FAST) ? q0 / p.gw : 0;
@@ -225,105 +227,109 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__
                 // warp has waited for every earlier stage before it reaches
                 // this one).
                 if (u == p.starve_step) break;
-                if (u >= S && !mbar_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag, p.wait_ns)) {
-                    fail(abort_flag, p.status, kStatusTimeoutProducer);
+                if (u >= S && !warp_wait(&bars[B_EMPTY + s], r_p ^ 1u, abort_flag, p.wait_ns)) {
+                    if (lane == 0) fail(abort_flag, p.status, kStatusTimeoutProducer);
                     break;
                 }
                 uint64_t* full = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(full, step_bytes + (pass_b ? v_bytes : 0u));
-                bulk_load(smem + L.k + s * L.k_bytes, p.kst + ((size_t)bh * T + t) * L.tile, L.tile, full);
-                if (BIAS == BIAS_RP_FAST) {
-                    // Entries xs .. xs + 255 of the reversed row for ri - rj,
-                    // xs = gw - 128 - (ci0 - cj0), from each shifted copy.
-                    const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
-                    const int rho = ri - rj + p.gh - 1;
-                    const int xs = p.gw - BM - (ci0 - cj0);
-                    const float* srcw = rps_h + (size_t)rho * 4 * row_len + xs;
-                    float* dst = reinterpret_cast<float*>(smem + L.rp) + (size_t)s * 4 * RP_STRIDE;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(full, step_bytes + (pass_b ? v_bytes : 0u));
+                    bulk_load(smem + L.k + s * L.k_bytes, p.kst + ((size_t)bh * T + t) * L.tile, L.tile, full);
+                    if (BIAS == BIAS_RP_FAST) {
+                        // Entries xs .. xs + 255 of the reversed row for ri - rj,
+                        // xs = gw - 128 - (ci0 - cj0), from each shifted copy.
+                        const int rj = j0 / p.gw, cj0 = j0 - rj * p.gw;
+                        const int rho = ri - rj + p.gh - 1;
+                        const int xs = p.gw - BM - (ci0 - cj0);
+                        const float* srcw = rps_h + (size_t)rho * 4 * row_len + xs;
+                        float* dst = reinterpret_cast<float*>(smem + L.rp) + (size_t)s * 4 * RP_STRIDE;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        bulk_load(dst + m * RP_STRIDE, srcw + m * row_len, RP_COPY_BYTES, full);
+                        for (int m = 0; m < 4; ++m)
+                            bulk_load(dst + m * RP_STRIDE, srcw + m * row_len, RP_COPY_BYTES, full);
+                    }
+                    if (BIAS == BA_BIAS_DENSE)
+                        for (int bx = 0; bx < 4; ++bx)
+                            tma_load_3d(smem + L.b + (s * 4 + bx) * 16384, &tm_b, full, j0 + 32 * bx, q0, h);
+                    if (pass_b)
+                        for (int vb = 0; vb < 2; ++vb)
+                            tma_load_3d(smem + L.v + (s * 2 + vb) * L.v_bytes, &tm_v, full, j0 + 64 * vb, 0, bh);
                 }
-                if (BIAS == BA_BIAS_DENSE)
-                    for (int bx = 0; bx < 4; ++bx)
-                        tma_load_3d(smem + L.b + (s * 4 + bx) * 16384, &tm_b, full, j0 + 32 * bx, q0, h);
-                if (pass_b)
-                    for (int vb = 0; vb < 2; ++vb)
-                        tma_load_3d(smem + L.v + (s * 2 + vb) * L.v_bytes, &tm_v, full, j0 + 64 * vb, 0, bh);
+                __syncwarp();
                 issued = u + 1;
             }
             // On an abort, let copies already issued land before the CTA exits.
-            if (*abort_flag)
+            if (__any_sync(0xffffffffu, *abort_flag != 0))
                 for (int u = (issued > S ? issued - S : 0); u < issued; ++u)
-                    mbar_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
+                    warp_wait(&bars[B_FULL + u % S], (u / S) & 1, nullptr, 100000000ull);
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------------- MMA issue
-        if (lane == 0) {
-            const uint32_t idesc_qk = (QK == QK_I8) ? instr_desc(kCS32, kFmtS8, kFmtS8, BM, BN)
-                                                    : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
-            const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
-            const uint32_t sbo_qk = (uint32_t)chunks * 128u;
-            bool ok = mbar_wait(&bars[B_QREADY], 0, abort_flag, p.wait_ns);
-            // Descriptors are built once; moving along a buffer only adds to the
-            // start-address field (bytes / 16), which never carries out.
-            const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
-            const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
-            const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
-            const uint32_t k_step = L.k_bytes >> 4, v_step = L.v_bytes >> 4;
-            const int kq = p.dpad / 32;
-            // QK of step u into S buffer u % NSB, once the softmax is done with
-            // the step that used it last (its PV, issued earlier, reads P
-            // before this product overwrites it: one thread's tcgen05 ops run
-            // in order).
-            // Stage and S buffer of the next QK (issued for steps in order):
-            // slot = step % ring size, parity = (step / ring size) & 1.
-            int q_s = 0, q_b = 0;
-            uint32_t q_sp = 0, q_bp = 0;
-            auto issue_qk = [&](int u) -> bool {
-                const int s = q_s, b = q_b;
-                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag, p.wait_ns)) return false;
-                if (u >= NSB && !mbar_wait(&bars[B_SDONE + b], q_bp ^ 1u, abort_flag, p.wait_ns)) return false;
+        // The whole warp runs this loop with uniform control flow and ring
+        // state; one elected lane issues each tensor-core instruction.
+        const uint32_t idesc_qk = (QK == QK_I8) ? instr_desc(kCS32, kFmtS8, kFmtS8, BM, BN)
+                                                : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
+        const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
+        const uint32_t sbo_qk = (uint32_t)chunks * 128u;
+        bool ok = warp_wait(&bars[B_QREADY], 0, abort_flag, p.wait_ns);
+        // Descriptors are built once; moving along a buffer only adds to the
+        // start-address field (bytes / 16), which never carries out.
+        const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
+        const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
+        const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
+        const uint32_t k_step = L.k_bytes >> 4, v_step = L.v_bytes >> 4;
+        const int kq = p.dpad / 32;
+        // QK of step u into S buffer u % NSB, once the softmax is done with
+        // the step that used it last (its PV, issued earlier, reads P before
+        // this product overwrites it: one thread's tcgen05 ops run in order).
+        // Stage and S buffer of the next QK (issued for steps in order):
+        // slot = step % ring size, parity = (step / ring size) & 1.
+        int q_s = 0, q_b = 0;
+        uint32_t q_sp = 0, q_bp = 0;
+        auto issue_qk = [&](int u) -> bool {
+            const int s = q_s, b = q_b;
+            if (!warp_wait(&bars[B_FULL + s], q_sp, abort_flag, p.wait_ns)) return false;
+            if (u >= NSB && !warp_wait(&bars[B_SDONE + b], q_bp ^ 1u, abort_flag, p.wait_ns)) return false;
+            tc_fence_after();
+            const uint64_t dk = dk0 + s * k_step;
+            const uint32_t d_tmem = tmem + b * BN;
+            for (int kk = 0; kk < kq; ++kk)
+                mma_ss_warp<QK>(d_tmem, dq0 + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
+            mma_commit_warp(&bars[B_SFULL + b]);
+            ring_next(q_s, q_sp, S);
+            ring_next(q_b, q_bp, NSB);
+            return true;
+        };
+        // QK runs LA steps ahead: two when four stages hold the key tiles of
+        // the steps in flight, else one.
+        const int LA = (S >= 4) ? 2 : 1;
+        for (int u = 0; ok && u < LA && u < U; ++u) ok = issue_qk(u);
+        int p_s = 0, p_b = 0;                      // stage and S buffer of step u
+        uint32_t p_sp = 0, p_bp = 0;
+        for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S), ring_next(p_b, p_bp, NSB)) {
+            if (u + LA < U && !(ok = issue_qk(u + LA))) break;
+            if (u >= T) {
+                // PV: u8 P x s8 V, K = 32 keys per product.  The P codes of
+                // keys 32 kq .. 32 kq + 31 sit in columns 32 kq .. 32 kq + 7 of
+                // the S buffer.
+                const int t = u - T, b = p_b, s = p_s;
+                if (!(ok = warp_wait(&bars[B_SDONE + b], p_bp, abort_flag, p.wait_ns))) break;
                 tc_fence_after();
-                const uint64_t dk = dk0 + s * k_step;
-                const uint32_t d_tmem = tmem + b * BN;
-                for (int kk = 0; kk < kq; ++kk)
-                    mma_ss<QK>(d_tmem, dq0 + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
-                mma_commit(&bars[B_SFULL + b]);
-                ring_next(q_s, q_sp, S);
-                ring_next(q_b, q_bp, NSB);
-                return true;
-            };
-            // QK runs LA steps ahead: two when four stages hold the key tiles
-            // of the steps in flight, else one.
-            const int LA = (S >= 4) ? 2 : 1;
-            for (int u = 0; ok && u < LA && u < U; ++u) ok = issue_qk(u);
-            int p_s = 0, p_b = 0;                  // stage and S buffer of step u
-            uint32_t p_sp = 0, p_bp = 0;
-            for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S), ring_next(p_b, p_bp, NSB)) {
-                if (u + LA < U && !(ok = issue_qk(u + LA))) break;
-                if (u >= T) {
-                    // PV: u8 P x s8 V, K = 32 keys per product.  The P codes of
-                    // keys 32 kq .. 32 kq + 31 sit in columns 32 kq .. 32 kq + 7
-                    // of the S buffer.
-                    const int t = u - T, b = p_b, s = p_s;
-                    if (!(ok = mbar_wait(&bars[B_SDONE + b], p_bp, abort_flag, p.wait_ns))) break;
-                    tc_fence_after();
-                    const uint32_t a_tmem = tmem + b * BN;
-                    for (int kk = 0; kk < BN / 32; ++kk)
-                        mma_ts_i8(tmem + O_COL, a_tmem + kk * KT,
-                                  dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
-                                  idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars[B_EMPTY + p_s]);
+                const uint32_t a_tmem = tmem + b * BN;
+#pragma unroll
+                for (int kk = 0; kk < BN / 32; ++kk)
+                    mma_ts_i8_warp(tmem + O_COL, a_tmem + kk * KT,
+                                   dv0 + (s * 2 + (kk >> 1)) * v_step + (kk & 1) * 2,
+                                   idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
             }
-            if (ok) mma_commit(&bars[B_OREADY]);
-            if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
-            // Let every issued MMA finish before TMEM is released.
-            mma_commit(&bars[B_FINAL]);
-            if (!mbar_wait(&bars[B_FINAL], 0, nullptr, 4000000000ull)) atomicOr(p.status, kStatusTimeoutMma);
+            mma_commit_warp(&bars[B_EMPTY + p_s]);
         }
+        if (ok) mma_commit_warp(&bars[B_OREADY]);
+        if (!ok && lane == 0) fail(abort_flag, p.status, kStatusTimeoutMma);
+        __syncwarp();
+        // Let every issued MMA finish before TMEM is released.
+        mma_commit_warp(&bars[B_FINAL]);
+        if (!warp_wait(&bars[B_FINAL], 0, nullptr, 4000000000ull) && lane == 0) atomicOr(p.status, kStatusTimeoutMma);
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax + epilogue

@@ -20,6 +20,7 @@
 // the kernel records a status bit, lets issued work drain, frees TMEM and
 // returns.
 #include "ba_attn_tc_common.cuh"
+#include "ba_tc_warp.cuh"
 
 namespace ba {
 namespace tc {
@@ -212,81 +213,83 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------------- MMA issue
-        if (lane == 0) {
-            const uint32_t idesc_qk = (QK == QK_I8) ? instr_desc(kCS32, kFmtS8, kFmtS8, BM, BN)
-                                                    : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
-            const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
-            const uint32_t sbo_qk = (uint32_t)chunks * 128u;
-            // Descriptors are built once; moving along a buffer only adds to the
-            // start-address field (bytes / 16), which never carries out.
-            const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
-            const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
-            const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
-            const uint32_t q_step = L.q_bytes >> 4, v_step = L.v_bytes >> 4;
-            const int kq = p.dpad / 32;
-            // Steps run on across tiles: the S buffer of global step w is w & 1,
-            // in its use (w >> 1); ring slots and parities are running counters.
-            int q_s = 0;                           // stage of the next QK
-            uint32_t q_sp = 0;
-            auto issue_qk = [&](int64_t w) -> bool {
-                const int s = q_s, buf = (int)(w & 1);
-                if (!mbar_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
-                for (int g = 0; g < NG; ++g)
-                    if (w >= 2 && !mbar_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)(((w >> 1) - 1) & 1), abort_flag))
-                        return false;
-                tc_fence_after();
-                for (int g = 0; g < NG; ++g) {
-                    const uint64_t dq = dq0 + g * q_step;
-                    const uint64_t dk = dk0 + ((s * L.k_bytes + g * L.tile) >> 4);
-                    const uint32_t d_tmem = tmem + (2 * g + buf) * BN;
-                    for (int kk = 0; kk < kq; ++kk)
-                        mma_ss<QK>(d_tmem, dq + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars[B_SFULL + 2 * g + buf]);
-                }
-                ring_next(q_s, q_sp, S);
-                return true;
-            };
-            bool ok = true;
-            int p_s = 0;                           // stage of the running step
-            uint32_t p_sp = 0;
-            int64_t gbase = 0;                     // global index of the tile's first step
-            int kt = 0;                            // tiles done by this CTA
-            for (int k = blockIdx.x; ok && k < p.tiles; k += gridDim.x, ++kt, gbase += U) {
-                // Q of this tile written by the softmax warps.
-                if (!(ok = mbar_wait(&bars[B_QREADY], (uint32_t)(kt & 1), abort_flag))) break;
-                if (!(ok = issue_qk(gbase))) break;
-                for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S)) {
-                    const int64_t w = gbase + u;
-                    if (u + 1 < U && !(ok = issue_qk(w + 1))) break;
-                    if (u >= T) {
-                        // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
-                        const int t = u - T, buf = (int)(w & 1), s = p_s;
-                        // The first PV of a tile overwrites the output accumulators:
-                        // the softmax warps must have read the previous tile's.
-                        if (t == 0 && kt > 0 &&
-                            !(ok = mbar_wait(&bars[B_OFREE], (uint32_t)((kt - 1) & 1), abort_flag)))
-                            break;
-                        for (int g = 0; g < NG && ok; ++g)
-                            ok = mbar_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)((w >> 1) & 1), abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        for (int g = 0; g < NG; ++g) {
-                            const uint64_t dv = dv0 + (s * KVG + g) * v_step;
-                            const uint32_t a_tmem = tmem + (2 * g + buf) * BN;
-                            for (int kk = 0; kk < BN / 32; ++kk)
-                                mma_ts_i8(tmem + 256 + 128 * g, a_tmem + kk * 8, dv + kk * 2, idesc_pv,
-                                          (t > 0 || kk > 0) ? 1u : 0u);
-                        }
-                    }
-                    mma_commit(&bars[B_EMPTY + p_s]);
-                }
-                if (ok) mma_commit(&bars[B_OREADY]);
+        // The whole warp runs this loop with uniform control flow and ring
+        // state; one elected lane issues each tensor-core instruction.
+        const uint32_t idesc_qk = (QK == QK_I8) ? instr_desc(kCS32, kFmtS8, kFmtS8, BM, BN)
+                                                : instr_desc(kCF32, kFmtE4M3, kFmtE4M3, BM, BN);
+        const uint32_t idesc_pv = instr_desc(kCS32, kFmtU8, kFmtS8, BM, p.dv);
+        const uint32_t sbo_qk = (uint32_t)chunks * 128u;
+        // Descriptors are built once; moving along a buffer only adds to the
+        // start-address field (bytes / 16), which never carries out.
+        const uint64_t dq0 = smem_desc(smem_addr(smem + L.q), 128, sbo_qk, kLayoutNone);
+        const uint64_t dk0 = smem_desc(smem_addr(smem + L.k), 128, sbo_qk, kLayoutNone);
+        const uint64_t dv0 = smem_desc(smem_addr(smem + L.v), 16, 512, kLayoutSw64);
+        const uint32_t q_step = L.q_bytes >> 4, v_step = L.v_bytes >> 4;
+        const int kq = p.dpad / 32;
+        // Steps run on across tiles: the S buffer of global step w is w & 1, in
+        // its use (w >> 1); ring slots and parities are running counters.
+        int q_s = 0;                               // stage of the next QK
+        uint32_t q_sp = 0;
+        auto issue_qk = [&](int64_t w) -> bool {
+            const int s = q_s, buf = (int)(w & 1);
+            if (!warp_wait(&bars[B_FULL + s], q_sp, abort_flag)) return false;
+            for (int g = 0; g < NG; ++g)
+                if (w >= 2 && !warp_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)(((w >> 1) - 1) & 1), abort_flag))
+                    return false;
+            tc_fence_after();
+            for (int g = 0; g < NG; ++g) {
+                const uint64_t dq = dq0 + g * q_step;
+                const uint64_t dk = dk0 + ((s * L.k_bytes + g * L.tile) >> 4);
+                const uint32_t d_tmem = tmem + (2 * g + buf) * BN;
+                for (int kk = 0; kk < kq; ++kk)
+                    mma_ss_warp<QK>(d_tmem, dq + kk * 16, dk + kk * 16, idesc_qk, kk > 0 ? 1u : 0u);
+                mma_commit_warp(&bars[B_SFULL + 2 * g + buf]);
             }
-            if (!ok) fail(abort_flag, p.status, kStatusTimeoutMma);
-            // Let every issued MMA finish before TMEM is released.
-            mma_commit(&bars[B_FINAL]);
-            if (!mbar_wait(&bars[B_FINAL], 0, nullptr, 4000000000ull)) atomicOr(p.status, kStatusTimeoutMma);
+            ring_next(q_s, q_sp, S);
+            return true;
+        };
+        bool ok = true;
+        int p_s = 0;                               // stage of the running step
+        uint32_t p_sp = 0;
+        int64_t gbase = 0;                         // global index of the tile's first step
+        int kt = 0;                                // tiles done by this CTA
+        for (int k = blockIdx.x; ok && k < p.tiles; k += gridDim.x, ++kt, gbase += U) {
+            // Q of this tile written by the softmax warps.
+            if (!(ok = warp_wait(&bars[B_QREADY], (uint32_t)(kt & 1), abort_flag))) break;
+            if (!(ok = issue_qk(gbase))) break;
+            for (int u = 0; ok && u < U; ++u, ring_next(p_s, p_sp, S)) {
+                const int64_t w = gbase + u;
+                if (u + 1 < U && !(ok = issue_qk(w + 1))) break;
+                if (u >= T) {
+                    // PV: u8 P (in the S buffer's first BN/4 TMEM columns) x s8 V.
+                    const int t = u - T, buf = (int)(w & 1), s = p_s;
+                    // The first PV of a tile overwrites the output accumulators:
+                    // the softmax warps must have read the previous tile's.
+                    if (t == 0 && kt > 0 &&
+                        !(ok = warp_wait(&bars[B_OFREE], (uint32_t)((kt - 1) & 1), abort_flag)))
+                        break;
+                    for (int g = 0; g < NG && ok; ++g)
+                        ok = warp_wait(&bars[B_SDONE + 2 * g + buf], (uint32_t)((w >> 1) & 1), abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int g = 0; g < NG; ++g) {
+                        const uint64_t dv = dv0 + (s * KVG + g) * v_step;
+                        const uint32_t a_tmem = tmem + (2 * g + buf) * BN;
+#pragma unroll
+                        for (int kk = 0; kk < BN / 32; ++kk)
+                            mma_ts_i8_warp(tmem + 256 + 128 * g, a_tmem + kk * 8, dv + kk * 2, idesc_pv,
+                                           (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit_warp(&bars[B_EMPTY + p_s]);
+            }
+            if (ok) mma_commit_warp(&bars[B_OREADY]);
         }
+        if (!ok && lane == 0) fail(abort_flag, p.status, kStatusTimeoutMma);
+        __syncwarp();
+        // Let every issued MMA finish before TMEM is released.
+        mma_commit_warp(&bars[B_FINAL]);
+        if (!warp_wait(&bars[B_FINAL], 0, nullptr, 4000000000ull) && lane == 0) atomicOr(p.status, kStatusTimeoutMma);
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
