@@ -16,6 +16,7 @@ import ctypes
 from . import _native as N
 
 __all__ = ["pack_qk", "quant_v", "prepass_qkv", "attention_fwd", "attention_fwd_noalloc", "attention_workspace",
+           "ForwardGraph",
            "workspace_bytes", "attention_bwd", "attention_decode", "scores_debug", "forward",
            "check_device_status", "words", "vq_ld"]
 
@@ -181,6 +182,70 @@ def attention_fwd(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NO
     _call(muq.device, "ba_attention_fwd_variant", _p(bq), _p(muq), _p(bk), _p(muk), _p(vq), _p(sv), kind, bp, ld,
           gh, gw, B, H, Nn, d, _p(workspace), ws_bytes, _p(out), _dt(out), int(variant), _stream(muq.device))
     return out
+
+
+class ForwardGraph:
+    """The forward hot path -- prepass_qkv(q, k, v) then attention_fwd -- for
+    fixed tensors, recorded once as a CUDA graph (ba_fwd_graph_create).
+    launch() queues one whole step on the current stream as a single graph
+    launch and returns `out`.  The object keeps a reference to every tensor
+    the graph reads or writes (q, k, v, the pre-pass outputs `pre`, `out`, the
+    bias and the workspace), so their storage outlives the graph; refill q, k
+    and v in place between steps.  `kernels` is the number of kernel
+    launches one step replays."""
+
+    def __init__(self, q, k, v, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None, out=None, out_dtype=None,
+                 variant=N.BA_QK_AUTO, pre=None, workspace=None):
+        torch = _torch()
+        self._h = None
+        _need_cuda(q, k, v)
+        B, H, Nn, d = q.shape
+        if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+            raise ValueError("q, k, v must share shape and dtype")
+        dev = q.device
+        if pre is None:
+            pre = (torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=dev),
+                   torch.empty((B, H, Nn), dtype=torch.float32, device=dev),
+                   torch.empty((B, H, Nn, words(d)), dtype=torch.int32, device=dev),
+                   torch.empty((B, H, Nn), dtype=torch.float32, device=dev),
+                   torch.empty((B, H, d, vq_ld(Nn)), dtype=torch.int8, device=dev),
+                   torch.empty((B, H, d), dtype=torch.float32, device=dev))
+        if out is None:
+            out = torch.empty((B, H, Nn, d), dtype=out_dtype or torch.float32, device=dev)
+        kind, bp, ld, gh, gw = _bias_args(bias, bias_kind, ld, grid)
+        if workspace is None:
+            if int(variant) not in (N.BA_QK_POPC, N.BA_QK_MMA_B1):
+                workspace = attention_workspace(B, H, Nn, d, kind, (gh, gw), device=dev)
+        else:
+            _need_cuda(workspace)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _same_device(q, k, v, *pre, out, workspace, bias)
+        bq, muq, bk, muk, vq, sv = pre
+        h = ctypes.c_void_p()
+        _call(dev, "ba_fwd_graph_create", _p(q), _p(k), _p(v), _dt(q), B, H, Nn, d, _p(bq), _p(muq), _p(bk),
+              _p(muk), _p(vq), _p(sv), kind, bp, ld, gh, gw, _p(workspace), ws_bytes, _p(out), _dt(out),
+              int(variant), ctypes.byref(h))
+        self._h = h
+        self._keep = (q, k, v, bias, workspace)
+        self.pre, self.out, self.device = pre, out, dev
+        self.kernels = int(N.lib().ba_fwd_graph_kernels(h))
+
+    def launch(self):
+        if self._h is None:
+            raise RuntimeError("ForwardGraph used after close()")
+        _call(self.device, "ba_fwd_graph_launch", self._h, _stream(self.device))
+        return self.out
+
+    def close(self):
+        if getattr(self, "_h", None) is not None:
+            N.check("ba_fwd_graph_destroy", N.lib().ba_fwd_graph_destroy(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def attention_fwd_noalloc(bq, muq, bk, muk, vq, sv, d, bias=None, bias_kind=N.BA_BIAS_NONE, ld=0, grid=None,

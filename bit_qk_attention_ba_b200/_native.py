@@ -36,6 +36,11 @@ SIGNATURES = {
                                       _P, _I, _I, _P]),
     "ba_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I, _P, _I,
                                       _P]),
+    "ba_fwd_graph_create": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I,
+                                 _P, _I64, _P, _I, _I, ctypes.POINTER(_P)]),
+    "ba_fwd_graph_launch": (_I, [_P, _P]),
+    "ba_fwd_graph_kernels": (_I, [_P]),
+    "ba_fwd_graph_destroy": (_I, [_P]),
     "ba_attention_bwd": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _I64, _I, _I, _I, _I, _I, _I,
                               _P, _P, ctypes.c_float, _P, _I64, _P, _P, _P, _P, _P]),
     "ba_attention_bwd_workspace_bytes": (_I64, [_I, _I, _I]),

@@ -110,12 +110,18 @@ static ba_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BA_OK : BA
 // queued on another device's stream would get the wrong ones.
 // BA_ERR_CUDA when the runtime cannot say (no device), BA_ERR_INVALID_ARG
 // when the stream belongs to another device.  Checked after every host-only
-// argument check, just before work is queued.
+// argument check, just before work is queued.  A stream that is being
+// captured into a CUDA graph cannot be asked for its device (the query would
+// invalidate the capture), so it is taken to be the current device's.
 ba_status check_stream(void* stream)
 {
     int cur = 0, sdev = 0;
     if (cudaGetDevice(&cur) != cudaSuccess) return BA_ERR_CUDA;
-    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) return BA_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) == cudaSuccess && cap != cudaStreamCaptureStatusNone) return BA_OK;
+    cudaGetLastError();
+    if (cudaStreamGetDevice(st, &sdev) != cudaSuccess) return BA_ERR_CUDA;
     return sdev == cur ? BA_OK : BA_ERR_INVALID_ARG;
 }
 

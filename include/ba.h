@@ -11,6 +11,9 @@
  *        channel-wise int8, integer PV product)
  *   FW   Overall framework (tiled attention in the FlashAttention2 style)
  *
+ * ba_graph.h (same conventions) declares the pre-pass + fused forward as one
+ * replayable CUDA graph.
+ *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
  *     in the layout stated and aligned to their element size; the int8 V codes
@@ -25,7 +28,10 @@
  *     word, SM count, the static scratch of ba_attention_fwd_noalloc) is that
  *     of the device current on the calling thread, and `stream` must belong
  *     to it (BA_ERR_INVALID_ARG otherwise; BA_ERR_CUDA when the runtime has
- *     no device).  The buffers must live on that device too.
+ *     no device).  The buffers must live on that device too.  A stream that
+ *     is being captured into a CUDA graph is taken to belong to the current
+ *     device (the runtime cannot be asked during a capture), so every entry
+ *     point may be recorded into a caller's own graph.
  *   - A launch failure reported by the CUDA runtime returns BA_ERR_CUDA.
  *   - Kernels that wait on hardware barriers give up after a bounded number of
  *     polls, record a code in a device status word and exit cleanly;

@@ -1,9 +1,10 @@
 """Host-side checks of the C ABI (no GPU needed, no compute calls).
 
-The library must load, export every function include/ba.h declares, and
+The library must load, export every function include/*.h declares, and
 reject invalid arguments before it touches the CUDA runtime.
 """
 import ctypes
+import glob
 import os
 import re
 
@@ -21,7 +22,7 @@ def lib():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "ba.h")).read()
+    src = "".join(open(p).read() for p in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(ba_[a-z_0-9]+)\s*\(", src)))
 
