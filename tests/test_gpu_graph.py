@@ -113,3 +113,38 @@ def test_graph_create_rejects_invalid_arguments():
     assert e.value.status == NAT.BA_ERR_INVALID_ARG
     torch.cuda.synchronize(dev)
     assert ba.check_device_status(dev) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["relaxed", "global"])
+def test_entry_points_record_into_a_callers_graph(mode):
+    """The eager calls recorded by the caller's own stream capture (torch's
+    CUDA graph) replay to the same results as running them directly."""
+    torch = _cuda()
+    import bit_qk_attention_ba_b200 as ba
+    dev = torch.device("cuda:0")
+    w = Workload("g_user", 2, 2, 197, 64, bias_std=0.3)
+    inp = make_inputs(w)
+    q, k, v = (torch.from_numpy(inp[n]).to(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+    bias = torch.from_numpy(inp["bias"]).to(dev)
+    kind, ld = BIAS_KIND[w.bias], inp["ld"]
+    pre = ba.prepass_qkv(q, k, v)
+    ws = ba.attention_workspace(w.B, w.H, w.N, w.d, kind, device=dev)
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    ba.attention_fwd(*pre, w.d, bias=bias, bias_kind=kind, ld=ld, out=out, workspace=ws)   # attributes set once
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode=mode):
+        ba.prepass_qkv(q, k, v, pre)
+        ba.attention_fwd(*pre, w.d, bias=bias, bias_kind=kind, ld=ld, out=out, workspace=ws)
+    nxt = make_inputs(w, seed=5)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        t.copy_(torch.from_numpy(nxt[name]).to(torch.bfloat16))
+    graph.replay()
+    got = out.clone()
+    pre_e = ba.prepass_qkv(q, k, v)
+    ref = ba.attention_fwd(*pre_e, w.d, bias=bias, bias_kind=kind, ld=ld, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize(dev)
+    assert torch.equal(got, ref)
+    assert ba.check_device_status(dev) == 0
+    del graph
