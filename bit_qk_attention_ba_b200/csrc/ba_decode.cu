@@ -75,6 +75,14 @@ __device__ __forceinline__ int dp4a_u8s8(uint32_t a_u8x4, uint32_t b_s8x4, int c
     return r;
 }
 
+// atomicAdd(ticket, 1) with release and acquire semantics at GPU scope.
+__device__ __forceinline__ unsigned ticket_acq_rel(unsigned* ticket)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
+    return old;
+}
+
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
@@ -240,22 +248,12 @@ decode_pv_kernel(const Params p)
     if (threadIdx.x < d)
         sm100::bulk_load(vt + (size_t)threadIdx.x * vst, p.vq + (bh * d + threadIdx.x) * p.ldv + j0,
                          (uint32_t)len16, &vbar);
-    load_queries<W>(p, bh, qs, cq);
-    if (threadIdx.x < p.Nq) {
-        float m = -INFINITY;
-        for (int t = 0; t < p.SA; ++t) m = fmaxf(m, p.pmax[(bh * p.SA + t) * p.Nq + threadIdx.x]);
-        negm[threadIdx.x] = -m * LOG2E;
-    }
-    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) sacc[e] = 0;
-    __syncthreads();
-    float l[NQ];
-#pragma unroll
-    for (int i = 0; i < NQ; ++i) l[i] = 0.f;
-    // KB keys per thread in flight: their loads first, then the codes.
+    // KB keys per thread in flight: their loads first, then the codes.  The
+    // first batch is loaded before the query side, so both round trips overlap.
     constexpr int KB = 4;
-    for (int jb = threadIdx.x; jb < len16; jb += KB * blockDim.x) {
-        uint32_t kb[KB][W];
-        float mk[KB];
+    uint32_t kb[KB][W];
+    float mk[KB];
+    auto load_batch = [&](int jb) {
 #pragma unroll
         for (int u = 0; u < KB; ++u) {
             const int jj = jb + u * blockDim.x;
@@ -267,6 +265,21 @@ decode_pv_kernel(const Params p)
                 mk[u] = __ldg(p.muk + bh * p.Nk + j0 + jj);
             }
         }
+    };
+    load_batch(threadIdx.x);
+    load_queries<W>(p, bh, qs, cq);
+    if (threadIdx.x < p.Nq) {
+        float m = -INFINITY;
+        for (int t = 0; t < p.SA; ++t) m = fmaxf(m, p.pmax[(bh * p.SA + t) * p.Nq + threadIdx.x]);
+        negm[threadIdx.x] = -m * LOG2E;
+    }
+    for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) sacc[e] = 0;
+    __syncthreads();
+    float l[NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) l[i] = 0.f;
+    for (int jb = threadIdx.x; jb < len16; jb += KB * blockDim.x) {
+        if (jb != (int)threadIdx.x) load_batch(jb);
 #pragma unroll
         for (int u = 0; u < KB; ++u) {
             const int jj = jb + u * blockDim.x;
@@ -333,13 +346,14 @@ decode_pv_kernel(const Params p)
 
     // The head's last split CTA to finish adds the splits (int64 code sums,
     // P~ sums in split order) and applies the epilogue O = sv acc / (255 l).
+    // The CTA's stores are ordered before thread 0's ticket by the barrier,
+    // and the ticket is a release (publishing them, cumulatively) and an
+    // acquire (the last CTA then sees every split's stores): one round trip.
     __shared__ unsigned s_last;
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&p.ticket[bh], 1u) == (unsigned)(p.S - 1);
+    if (threadIdx.x == 0) s_last = ticket_acq_rel(&p.ticket[bh]) == (unsigned)(p.S - 1);
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     for (int e = threadIdx.x; e < p.Nq * d; e += blockDim.x) {
         const int i = e / d, c2 = e - i * d;
         long long tot = 0;
