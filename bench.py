@@ -336,29 +336,37 @@ def time_side_workload(w, variant, dev, steps=50, warmup=10):
     step_ms = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
     attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
     # The same step replayed from one CUDA graph (ba_fwd_graph_*): its kernels
-    # run back to back, without a host launch per kernel.
-    graph = ba.ForwardGraph(q, k, v, bias=bias, bias_kind=kind, ld=ld, grid=grid, out_dtype=tdt, variant=variant)
-    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    for _ in range(warmup):
-        graph.launch()
-    torch.cuda.synchronize(dev)
-    for i in range(steps):
-        if flush is not None:
-            flush.zero_()
-        gev[i][0].record(stream)
-        graph.launch()
-        gev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    graph_ms = statistics.median(a.elapsed_time(b) for a, b in gev)
-    graph_kernels = graph.kernels
-    graph.close()
+    # run back to back, without a host launch per kernel.  A failure to build
+    # the graph is reported in the line instead of ending the run.
+    graph, graph_ms, graph_kernels, graph_error = None, None, None, None
+    try:
+        graph = ba.ForwardGraph(q, k, v, bias=bias, bias_kind=kind, ld=ld, grid=grid, out_dtype=tdt,
+                                variant=variant)
+    except Exception as e:          # noqa: BLE001 -- recorded in the JSON line
+        graph_error = str(e)
+    if graph is not None:
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for _ in range(warmup):
+            graph.launch()
+        torch.cuda.synchronize(dev)
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            gev[i][0].record(stream)
+            graph.launch()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = statistics.median(a.elapsed_time(b) for a, b in gev)
+        graph_kernels = graph.kernels
+        graph.close()
     roof = roofline(w, attn_ms * 1e-3, 2 if tdt == torch.bfloat16 else 4, variant)
     status = ba.check_device_status(dev)
     del q, k, v, bias, pre, out, ws, flush, graph
     torch.cuda.empty_cache()
     return {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "bias": w.bias, "attention_us": attn_ms * 1e3,
             "step_us": step_ms * 1e3, "step_tops": w.ops / (step_ms * 1e-3) / 1e12,
-            "graph_step_us": graph_ms * 1e3, "graph_kernels": graph_kernels,
+            "graph_step_us": None if graph_ms is None else graph_ms * 1e3, "graph_kernels": graph_kernels,
+            **({"graph_error": graph_error} if graph_error else {}),
             "attention_tops": w.ops / (attn_ms * 1e-3) / 1e12, "steps": steps, "warmup": warmup,
             "l2": "flushed between steps" if in_bytes < 2 * L2_BYTES else "inputs larger than L2",
             "roofline": roof, "device_status": status}
