@@ -47,8 +47,13 @@ def _p(t):
 def _call(device, fn, *args):
     """Call a libba entry point with `device` current: the library looks up
     its per-device state (status word, SM count, static scratch) on the
-    current device, and rejects a stream that belongs to another one."""
+    current device, and rejects a stream that belongs to another one.  The
+    device is switched only when another one is current (the switch costs a
+    few microseconds of host time per call)."""
     torch = _torch()
+    if device.index is None or torch.cuda.current_device() == device.index:
+        N.call(fn, *args)
+        return
     with torch.cuda.device(device):
         N.call(fn, *args)
 
